@@ -82,6 +82,7 @@ typedef enum eagle_attn_status {
 #define EAGLE_ATTN_DEV_POS_OUTSIDE 3      /* a query or key position lies past cu_seqlens[num_docs] */
 #define EAGLE_ATTN_DEV_TIMEOUT 4          /* a pipeline wait gave up (a library bug; no input causes it) */
 #define EAGLE_ATTN_DEV_BAD_TILE 5         /* a q_tiles entry is negative, >= Tq or not a multiple of 128 */
+#define EAGLE_ATTN_DEV_SMEM_ALIGN 6       /* dynamic shared memory not 1024-byte aligned (a library bug) */
 
 typedef enum eagle_attn_dtype {
     EAGLE_ATTN_F32 = 0,
@@ -115,7 +116,12 @@ typedef struct eagle_attn_params {
     int32_t B, Tq, Tk, H, D;   /* Tk = block-0 key length; num_blocks > 1 requires Tk == Tq */
     int32_t num_blocks;        /* NB >= 1: block 0 + (NB - 1) diagonal blocks */
     int32_t causal;            /* 1: key position <= query position (default); 0: no position mask */
-    int32_t deterministic;     /* backward: 1 = bitwise reproducible (no atomics) */
+    int32_t deterministic;     /* backward, tensor-core path: 0 (default) = one dK/dV/dQ kernel,
+                                  five products per tile pair, dQ summed with fp32 atomics (the
+                                  order of the additions, so the last bits of dq, vary from run
+                                  to run); 1 = bitwise reproducible: a dK/dV kernel and a dQ
+                                  kernel (which recomputes S and dP), no atomics.  The CUDA-core
+                                  path is always reproducible. */
     float scale;               /* softmax scale (typically D^-0.5) */
     int64_t q_pos_offset;      /* global position of query row 0 */
     int64_t k_pos_offset;      /* global position of block-0 key 0 */

@@ -24,7 +24,8 @@ STATUS = {
 NOALLOC_SCRATCH_BYTES = 32 << 20
 DEV_STATUS = {0: "EAGLE_ATTN_DEV_OK", 1: "EAGLE_ATTN_DEV_BAD_CU_SEQLENS",
               2: "EAGLE_ATTN_DEV_DOC_TOO_LONG", 3: "EAGLE_ATTN_DEV_POS_OUTSIDE",
-              4: "EAGLE_ATTN_DEV_TIMEOUT", 5: "EAGLE_ATTN_DEV_BAD_TILE"}
+              4: "EAGLE_ATTN_DEV_TIMEOUT", 5: "EAGLE_ATTN_DEV_BAD_TILE",
+              6: "EAGLE_ATTN_DEV_SMEM_ALIGN"}
 
 F32, BF16 = 0, 1
 GRAD_STORE, GRAD_ACCUMULATE_F32 = 0, 1

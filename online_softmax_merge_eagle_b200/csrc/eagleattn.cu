@@ -3,6 +3,7 @@
 // kernels and the generic CUDA-core kernels, and launches.  One translation
 // unit: the kernel headers below are included here.
 #include <cuda_runtime.h>
+#include <stdint.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -198,43 +199,6 @@ int tc_fwd_launch(const Problem &P, const eagle_attn_params *p, cudaStream_t s) 
     return EAGLE_ATTN_ERR_UNSUPPORTED;
 }
 
-template <int D>
-int tc_bwd_run(const Problem &P, const eagle_attn_params *p, const float *Dws,
-               const float *dq_diag, cudaStream_t s) {
-    namespace kv = tcbwd::kv;
-    namespace qk = tcbwd::qk;
-    static_assert(kv::BM == qk::BM && kv::BN == qk::BN && kv::BM == kv::BN,
-                  "both backward kernels share one set of 128-row tensor maps");
-    CUtensorMap tq, tdo, tk, tv;
-    if (!make_q_tmap(&tq, p->q, P, kv::BM) || !make_q_tmap(&tdo, p->grad_out, P, kv::BM) ||
-        !make_kv_tmap(&tk, p->cache_k, P, kv::BN) || !make_kv_tmap(&tv, p->cache_v, P, kv::BN))
-        return EAGLE_ATTN_ERR_CUDA;
-    auto k1 = kv::dkdv_kernel<D>;
-    auto k2 = qk::dq_kernel<D>;
-    const int s1 = kv::Cfg<D>::SMEM, s2 = qk::Cfg<D>::SMEM;
-    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess ||
-        cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess)
-        return EAGLE_ATTN_ERR_CUDA;
-    typedef __nv_bfloat16 bf;
-    prof_mark(p->prof_start, s);
-    dim3 g1((P.Tk + kv::BN - 1) / kv::BN, P.H, P.B);
-    k1<<<g1, tcbwd::THREADS, s1, s>>>(tq, tdo, tk, tv, P, p->lse, Dws, p->dk, p->dv);
-    if (after_launch()) return EAGLE_ATTN_ERR_CUDA;
-    dim3 g2((P.Tq + qk::BM - 1) / qk::BM, P.H, P.B);
-    k2<<<g2, tcbwd::THREADS, s2, s>>>(tq, tdo, tk, tv, P, p->lse, Dws, dq_diag, p->dq);
-    int rc = after_launch();
-    prof_mark(p->prof_stop, s);
-    return rc;
-}
-
-int tc_bwd_launch(const Problem &P, const eagle_attn_params *p, const float *Dws,
-                  const float *dq_diag, cudaStream_t s) {
-    if (P.Tq == 0 && P.Tk == 0) return EAGLE_ATTN_OK;
-    if (P.D == 128) return tc_bwd_run<128>(P, p, Dws, dq_diag, s);
-    if (P.D == 64) return tc_bwd_run<64>(P, p, Dws, dq_diag, s);
-    return EAGLE_ATTN_ERR_UNSUPPORTED;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWorkspace {
@@ -254,6 +218,85 @@ BwdWorkspace carve(const Problem &P, void *ws) {
 }
 
 int64_t rows_of(const Problem &P) { return (int64_t)P.B * P.Tq * P.H; }
+
+// dq = scale * dq_acc (fp32 [B, H, Tq, D]) in dq's dtype, or added to an fp32 dq.
+template <int D>
+int dq_finalize_launch(const Problem &P, const eagle_attn_params *p, const float *dq_acc,
+                       cudaStream_t s) {
+    constexpr int E = D / 32;
+    const int64_t rows = rows_of(P);
+    if (rows == 0) return EAGLE_ATTN_OK;
+    dim3 grid((unsigned)((rows + 7) / 8));
+    if (P.grad_accum)
+        dq_finalize_kernel<float, E><<<grid, ROW_THREADS, 0, s>>>(P, dq_acc, (float *)p->dq);
+    else
+        dq_finalize_kernel<__nv_bfloat16, E><<<grid, ROW_THREADS, 0, s>>>(
+            P, dq_acc, (__nv_bfloat16 *)p->dq);
+    return after_launch();
+}
+
+template <int D>
+int tc_bwd_run(const Problem &P, const eagle_attn_params *p, const float *Dws, float *dq_acc,
+               bool has_diag, cudaStream_t s) {
+    namespace kv = tcbwd::kv;
+    namespace qk = tcbwd::qk;
+    namespace kvq = tcbwd::kvq;
+    static_assert(kv::BM == qk::BM && kv::BN == qk::BN && kv::BM == kv::BN &&
+                      kvq::BM == kv::BM && kvq::BN == kv::BN,
+                  "the backward kernels share one set of 128-row tensor maps");
+    CUtensorMap tq, tdo, tk, tv;
+    if (!make_q_tmap(&tq, p->q, P, kv::BM) || !make_q_tmap(&tdo, p->grad_out, P, kv::BM) ||
+        !make_kv_tmap(&tk, p->cache_k, P, kv::BN) || !make_kv_tmap(&tv, p->cache_v, P, kv::BN))
+        return EAGLE_ATTN_ERR_CUDA;
+    if (!p->deterministic) {
+        // one kernel, five products per tile pair; dQ summed in dq_acc (which the
+        // row pass initialised), then scaled into dq
+        // the accumulator [B, H, Tq, D] as rows x D, in the reduce-add boxes
+        const int64_t acc_rows = (int64_t)P.B * P.H * P.Tq;
+        if (acc_rows + kvq::BM > INT32_MAX) return EAGLE_ATTN_ERR_SHAPE;
+        CUtensorMap tdq;
+        if (!make_tmap_f32_2d(&tdq, dq_acc, (uint64_t)D, (uint64_t)acc_rows, kvq::DQ_BOX_COLS,
+                              kvq::DQ_BOX_ROWS))
+            return EAGLE_ATTN_ERR_CUDA;
+        auto k = kvq::dkdvdq_kernel<D>;
+        const int sm = kvq::Cfg<D>::SMEM;
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
+            cudaSuccess)
+            return EAGLE_ATTN_ERR_CUDA;
+        prof_mark(p->prof_start, s);
+        dim3 g((P.Tk + kvq::BN - 1) / kvq::BN, P.H, P.B);
+        k<<<g, tcbwd::THREADS, sm, s>>>(tq, tdo, tk, tv, tdq, P, p->lse, Dws, p->dk, p->dv);
+        if (after_launch()) return EAGLE_ATTN_ERR_CUDA;
+        int rc = dq_finalize_launch<D>(P, p, dq_acc, s);
+        prof_mark(p->prof_stop, s);
+        return rc;
+    }
+    const float *dq_diag = has_diag ? dq_acc : nullptr;
+    auto k1 = kv::dkdv_kernel<D>;
+    auto k2 = qk::dq_kernel<D>;
+    const int s1 = kv::Cfg<D>::SMEM, s2 = qk::Cfg<D>::SMEM;
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess ||
+        cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess)
+        return EAGLE_ATTN_ERR_CUDA;
+    typedef __nv_bfloat16 bf;
+    prof_mark(p->prof_start, s);
+    dim3 g1((P.Tk + kv::BN - 1) / kv::BN, P.H, P.B);
+    k1<<<g1, tcbwd::THREADS, s1, s>>>(tq, tdo, tk, tv, P, p->lse, Dws, p->dk, p->dv);
+    if (after_launch()) return EAGLE_ATTN_ERR_CUDA;
+    dim3 g2((P.Tq + qk::BM - 1) / qk::BM, P.H, P.B);
+    k2<<<g2, tcbwd::THREADS, s2, s>>>(tq, tdo, tk, tv, P, p->lse, Dws, dq_diag, p->dq);
+    int rc = after_launch();
+    prof_mark(p->prof_stop, s);
+    return rc;
+}
+
+int tc_bwd_launch(const Problem &P, const eagle_attn_params *p, const float *Dws, float *dq_acc,
+                  bool has_diag, cudaStream_t s) {
+    if (P.Tq == 0 && P.Tk == 0) return EAGLE_ATTN_OK;
+    if (P.D == 128) return tc_bwd_run<128>(P, p, Dws, dq_acc, has_diag, s);
+    if (P.D == 64) return tc_bwd_run<64>(P, p, Dws, dq_acc, has_diag, s);
+    return EAGLE_ATTN_ERR_UNSUPPORTED;
+}
 
 template <typename T, typename TO, int E>
 int bwd_prep_launch(const Problem &P, const eagle_attn_params *p, BwdWorkspace w, cudaStream_t s) {
@@ -313,23 +356,25 @@ int bwd_all(const Problem &P, const eagle_attn_params *p, bool tc, cudaStream_t 
     BwdWorkspace w = carve(P, p->workspace);
     if (tc) {
         // tensor-core path: one row pass (D_t, diagonal grads, sum_i dz_i k_i
-        // into the dQ workspace), then dkdv_kernel and dq_kernel
+        // into the dQ workspace, zeros there without diagonal blocks when the
+        // five-product kernel adds into it), then the block-0 kernels
         const int64_t rows = rows_of(P);
+        const int zero_dq = p->deterministic ? 0 : 1;
         if (rows > 0) {
             dim3 grid((unsigned)((rows + 7) / 8));
             if (P.grad_accum)
                 bwd_rows_kernel<T, TO, float, E><<<grid, ROW_THREADS, 0, s>>>(
                     P, (const T *)p->q, (const T *)p->cache_k, (const T *)p->cache_v,
                     (const T *)p->grad_out, (const TO *)p->out, p->lse, w.Dt, w.dq_acc,
-                    (float *)p->dk, (float *)p->dv);
+                    (float *)p->dk, (float *)p->dv, zero_dq);
             else
                 bwd_rows_kernel<T, TO, T, E><<<grid, ROW_THREADS, 0, s>>>(
                     P, (const T *)p->q, (const T *)p->cache_k, (const T *)p->cache_v,
                     (const T *)p->grad_out, (const TO *)p->out, p->lse, w.Dt, w.dq_acc,
-                    (T *)p->dk, (T *)p->dv);
+                    (T *)p->dk, (T *)p->dv, zero_dq);
             if (after_launch()) return EAGLE_ATTN_ERR_CUDA;
         }
-        return tc_bwd_launch(P, p, w.Dt, P.NB > 1 ? w.dq_acc : nullptr, s);
+        return tc_bwd_launch(P, p, w.Dt, w.dq_acc, P.NB > 1, s);
     }
     int rc = bwd_prep_launch<T, TO, E>(P, p, w, s);
     if (rc) return rc;
@@ -532,15 +577,19 @@ int noalloc_scratch(void **out) {
 extern "C" {
 
 int eagle_attn_bwd_noalloc(const eagle_attn_params *p, void *stream) {
+    if (!p) return EAGLE_ATTN_ERR_NULL;
+    // the caller's workspace fields are ignored: validate without them
+    eagle_attn_params q = *p;
+    q.workspace = nullptr;
+    q.workspace_bytes = 0;
     Resolved r;
-    int rc = resolve(p, true, &r);
+    int rc = resolve(&q, true, &r);
     if (rc) return rc;
     if (bwd_ws_bytes(r.P) > (size_t)EAGLE_ATTN_NOALLOC_SCRATCH_BYTES)
         return EAGLE_ATTN_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
     rc = noalloc_scratch(&scratch);
     if (rc) return rc;
-    eagle_attn_params q = *p;
     q.workspace = scratch;
     q.workspace_bytes = EAGLE_ATTN_NOALLOC_SCRATCH_BYTES;
     return eagle_attn_bwd(&q, stream);

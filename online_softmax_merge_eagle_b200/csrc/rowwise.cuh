@@ -5,6 +5,7 @@
 //   bwd_prep_kernel       D_t = dO_t . O_t, zero the dQ accumulator
 //   bwd_diag_kernel       diagonal dq/dk/dv in closed form + dq write-out
 //   bwd_rows_kernel       D_t, diagonal dk/dv and sum_i dz_i k_i for the tensor-core backward
+//   dq_finalize_kernel    dq = scale * the fp32 dQ accumulator (five-product backward)
 //   wait_timeout_selftest_kernel   the bounded pipeline wait giving up (self-test)
 // Rows are (b, t, h) triples; row r of a contiguous [B, T, H, D] tensor starts
 // at r * D, and its lse sits at (b * H + h) * T + t.
@@ -333,13 +334,14 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_diag_kernel(
 // (dq_diag, fp32 [B, H, Tq, D]).  (NeMo AutoModel "eagle.ring_attention",
 // _CachedRingAttention: "the diagonal grads are added in closed form".)
 // dk / dv of the diagonal blocks in GT: T (written), or fp32 with P.grad_accum
-// (added to what the buffers hold).
+// (added to what the buffers hold).  With zero_dq, dq_diag is written (zeros)
+// also when there are no diagonal blocks.
 template <typename T, typename TO, typename GT, int E>
 __global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
     Problem P, const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ dout, const TO *__restrict__ out, const float *__restrict__ lse,
     float *__restrict__ Dws, float *__restrict__ dq_diag, GT *__restrict__ dk,
-    GT *__restrict__ dv) {
+    GT *__restrict__ dv, int zero_dq) {
     int64_t row = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= (int64_t)P.B * P.Tq * P.H) return;
@@ -356,7 +358,14 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
     for (int e = 0; e < E; ++e) part = fmaf(g[e], o[e], part);
     const float Dt = warp_sum(part);
     if (lane == 0) Dws[li] = Dt;
-    if (P.NB < 2) return;
+    if (P.NB < 2) {
+        if (zero_dq) {  // the accumulator the five-product backward adds into
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = 0.f;
+            RowIO<float, E>::store(dq_diag + li * P.D + lane * E, acc);
+        }
+        return;
+    }
     RowIO<T, E>::load(q + qo, qf);
     const float L = lse[li];
 #pragma unroll
@@ -396,6 +405,35 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
         RowIO<GT, E>::store(dv + ko, gv);
     }
     RowIO<float, E>::store(dq_diag + li * P.D + lane * E, acc);
+}
+
+// dq_t = scale * dq_acc_t, the fp32 accumulator ([B, H, Tq, D]) that the
+// five-product backward added its dS K products to (it started from the
+// diagonal blocks' sum_i dz_i k_i): written in GT, or added to the fp32 dq
+// with P.grad_accum.
+template <typename GT, int E>
+__global__ void __launch_bounds__(ROW_THREADS) dq_finalize_kernel(Problem P,
+                                                                 const float *__restrict__ dq_acc,
+                                                                 GT *__restrict__ dq) {
+    int64_t row = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= (int64_t)P.B * P.Tq * P.H) return;
+    const int h = (int)(row % P.H);
+    const int t = (int)((row / P.H) % P.Tq);
+    const int b = (int)(row / ((int64_t)P.H * P.Tq));
+    const int64_t qo = b * P.q_sb + t * P.q_st + (int64_t)h * P.D + lane * E;
+    const int64_t li = ((int64_t)b * P.H + h) * P.Tq + t;
+    float a[E];
+    RowIO<float, E>::load(dq_acc + li * P.D + lane * E, a);
+#pragma unroll
+    for (int e = 0; e < E; ++e) a[e] *= P.scale;
+    if (P.grad_accum) {
+        float o[E];
+        RowIO<GT, E>::load(dq + qo, o);
+#pragma unroll
+        for (int e = 0; e < E; ++e) a[e] += o[e];
+    }
+    RowIO<GT, E>::store(dq + qo, a);
 }
 
 // One warp waits, with the pipelines' bounded wait, on an mbarrier nothing

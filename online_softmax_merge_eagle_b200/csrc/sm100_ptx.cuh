@@ -96,6 +96,29 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const void *tmap, uint64_
         : "memory");
 }
 
+// Element-wise add of a shared-memory box into the global tensor `tmap`
+// describes (fp32 reduce-add, performed at L2 in whole lines); box origin at
+// (c0 = innermost, c1).  Part of the issuing thread's current bulk group.
+__device__ __forceinline__ void tma_reduce_add_2d(const void *tmap, const void *src, int c0,
+                                                  int c1) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], "
+        "[%1];" ::"l"(tmap),
+        "r"(smem_u32(src)), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until every bulk group of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until every bulk group of this thread has completed (writes included).
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // -------------------------------------------------------------- tcgen05 --
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -243,10 +266,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     return d;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D; A K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+// Instruction descriptor of kind::f16 with bf16 A/B, fp32 D; A K-major unless
+// a_mn_major (bit 15), B K-major unless b_mn_major (bit 16).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major,
+                                                  bool a_mn_major = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
 }
 
 // Byte offset of the 16-byte chunk `c` of row `r` in a [rows x (8*nchunks*...)]
@@ -260,19 +286,6 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// Per-warpgroup register budget (all four warps of the warpgroup execute it):
-// dec hands registers back to the CTA's pool, inc takes them from it.  The
-// increments of a kernel must fit in what its launch reserved (threads x
-// registers per thread at launch), or inc waits forever.
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {

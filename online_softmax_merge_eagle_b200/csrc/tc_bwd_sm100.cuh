@@ -719,6 +719,445 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 }  // namespace qk
+
+// ========================================================= dK / dV / dQ ===
+// The backward with five products per tile pair (the non-deterministic
+// mode): one CTA per 128 keys steps over 128-row query slices as
+// kv::dkdv_kernel does and, from the dS^T tile it already holds, also forms
+// dQ_i = dS_i K (M = 128 rows, N = D, K = the CTA's 128 keys), which it adds
+// to the fp32 dQ accumulator in global memory (the order of those fp32
+// additions across CTAs varies from run to run).  dS^T goes to shared memory
+// once, bf16 with the 128-byte swizzle, and serves as the K-major A operand of
+// dK += dS^T Q and as the MN-major A operand of dQ_i = dS K.  dQ_i leaves
+// through the same shared tile once both products have read it: two halves of
+// 64 rows, staged in the swizzled boxes of a TMA tensor map over the
+// accumulator and added there by TMA reduce-adds (whole L2 lines, a handful
+// of requests per slice instead of one per 16 bytes and thread).
+// TMEM: dV [0, D), dK [128, 128 + D) and two 128-column regions R0, R1 that
+// carry in turn S^T_i -> P^T_i (R_{i%2}), dP^T_i (R_{(i+1)%2}) and dQ_i
+// (R_{i%2}, issued after dV_i has read P^T_i).
+// MMA issue order: S^T_0, dP^T_0, then per step i: dV_i (once P^T_i is
+// written); S^T_{i+1}, dK_i, dQ_i (once dS^T_i is in shared memory);
+// dP^T_{i+1} (once the element-wise warps have read dQ_i out of R_{i%2}).
+// Element-wise order per step: P^T_i, then dQ_{i-1} out to global memory,
+// then dS^T_i.  Every wait of the element-wise warps is ANDed over all of
+// them (a named barrier), so they take every exit decision together.
+namespace kvq {
+
+constexpr int BN = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dV, dK)
+constexpr int BM = 128;  // query rows per step (TMEM lanes of dQ_i)
+constexpr int QS = 2;    // Q / dO ring depth
+constexpr int DQ_BOX_COLS = 32;  // fp32 box of the dQ tensor map: 32 columns (128 bytes)
+constexpr int DQ_BOX_ROWS = 64;  // x 64 rows (half a slice)
+
+template <int D>
+struct Cfg {
+    static constexpr int KT = BN * D * 2;    // K or V tile bytes
+    static constexpr int QT = BM * D * 2;    // Q or dO slice bytes
+    static constexpr int DST = BN * BM * 2;  // dS^T tile bytes (also the dQ staging)
+    static_assert(DQ_BOX_ROWS * D * 4 <= DST, "a half dQ slice fits the dS^T tile");
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KT;
+    static constexpr int OFF_Q = OFF_V + KT;
+    static constexpr int OFF_DO = OFF_Q + QS * QT;
+    static constexpr int OFF_DS = OFF_DO + QS * QT;
+    static constexpr int OFF_ROW = OFF_DS + DST;  // lse2[BM], D[BM], lo[BM], hi[BM], 2 ints
+    static constexpr int ROW_BYTES = 4 * BM * 4 + 16;
+    static constexpr int OFF_BAR = OFF_ROW + ROW_BYTES;
+    static constexpr int NBARS = 12;  // >= the barriers laid out in the kernel
+    // no realignment slack: the kernel checks that the base is 1024-byte aligned
+    static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16;
+    static_assert(SMEM <= 232448, "shared memory");
+    static constexpr uint32_t T_DV = 0, T_DK = 128, T_R0 = 256, T_R1 = 384, TMEM_COLS = 512;
+    static_assert(D <= 128, "TMEM budget");
+};
+
+// Named barrier 2 over the element-wise warps.
+__device__ __forceinline__ void ew_sync() {
+    asm volatile("bar.sync 2, %0;" ::"n"(EW_THREADS) : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1)
+    dkdvdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_dq, const Problem P,
+                  const float *__restrict__ lse, const float *__restrict__ Dws,
+                  void *__restrict__ dk, void *__restrict__ dv) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw;
+    // the swizzled tiles need a 1024-byte aligned base (CTA-uniform test; nothing
+    // has been allocated or started yet)
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) raise_status(EAGLE_ATTN_DEV_SMEM_ALIGN);
+        return;
+    }
+    uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
+    uint64_t *bar_kv = bars + 0;
+    uint64_t *bar_qf = bars + 1, *bar_qe = bars + 1 + QS;  // QS each
+    uint64_t *bar_sf = bars + 1 + 2 * QS;  // S^T_i in TMEM
+    uint64_t *bar_dpf = bar_sf + 1;        // dP^T_i in TMEM
+    uint64_t *bar_dqf = bar_dpf + 1;       // dQ_i in TMEM (dK_i done too: dS^T free)
+    uint64_t *bar_ptf = bar_dqf + 1;       // P^T_i written over S^T_i (EW_THREADS)
+    uint64_t *bar_dsf = bar_ptf + 1;       // dS^T_i in shared memory, dP^T_i read (EW_THREADS)
+    uint64_t *bar_dqe = bar_dsf + 1;       // dQ_i read out of TMEM (EW_THREADS)
+    uint64_t *bar_done = bar_dqe + 1;
+    static_assert(C::NBARS >= 1 + 2 * QS + 7, "barrier slots");
+    uint32_t *tmem_slot = (uint32_t *)(bars + C::NBARS);
+    volatile int *abort = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ks = blockIdx.x * BN, h = blockIdx.y, b = blockIdx.z;
+    int tbeg, tend;
+    keys_row_range(P.mask, ks, min(ks + BN, P.Tk) - 1, tbeg, tend);
+    const int nsteps = tend >= tbeg ? (tend - tbeg + BM) / BM : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NBARS; ++i) mbar_init(&bars[i], 1);
+        mbar_init(bar_ptf, EW_THREADS);
+        mbar_init(bar_dsf, EW_THREADS);
+        mbar_init(bar_dqe, EW_THREADS);
+        *abort = status_bad() ? 1 : 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool skip = *abort != 0;
+    // region of S^T_i / P^T_i / dQ_i (i even: R0); dP^T_i takes region(i + 1)
+    auto region = [&](int i) -> uint32_t { return (i & 1) ? C::T_R1 : C::T_R0; };
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0 && !skip) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_do);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            mbar_expect_tx(bar_kv, 2 * C::KT);
+#pragma unroll
+            for (int cb = 0; cb < D / 64; ++cb) {
+                tma_load_5d(smem + C::OFF_K + cb * BN * 128, &tm_k, bar_kv, cb * 64, h, ks, 0, b);
+                tma_load_5d(smem + C::OFF_V + cb * BN * 128, &tm_v, bar_kv, cb * 64, h, ks, 0, b);
+            }
+            int issued = 0;
+            for (int i = 0; i < nsteps; ++i) {
+                const int st = i % QS;
+                const int t0 = tbeg + i * BM;
+                if (!mbar_wait(bar_qe + st, ((i / QS) & 1) ^ 1, abort)) break;
+                mbar_expect_tx(bar_qf + st, 2 * C::QT);
+#pragma unroll
+                for (int cb = 0; cb < D / 64; ++cb) {
+                    tma_load_4d(smem + C::OFF_Q + st * C::QT + cb * BM * 128, &tm_q, bar_qf + st,
+                                cb * 64, h, t0, b);
+                    tma_load_4d(smem + C::OFF_DO + st * C::QT + cb * BM * 128, &tm_do, bar_qf + st,
+                                cb * 64, h, t0, b);
+                }
+                issued = i + 1;
+            }
+            if (*abort) {
+                drain_wait(bar_kv, 0);
+                for (int i = (issued > QS ? issued - QS : 0); i < issued; ++i)
+                    drain_wait(bar_qf + i % QS, (i / QS) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA ---
+        if (lane == 0 && !skip) {
+            const uint32_t id_st = idesc_bf16(BN, BM, false);      // M = 128 keys, N = 128 rows
+            const uint32_t id_acc = idesc_bf16(BN, D, true);       // M = 128 keys, N = D, B MN-major
+            const uint32_t id_dq = idesc_bf16(BM, D, true, true);  // M = 128 rows, N = D, A, B MN-major
+            const uint32_t k_s = smem_u32(smem + C::OFF_K), v_s = smem_u32(smem + C::OFF_V);
+            const uint32_t q_s = smem_u32(smem + C::OFF_Q), do_s = smem_u32(smem + C::OFF_DO);
+            const uint32_t ds_s = smem_u32(smem + C::OFF_DS);
+            bool ok = mbar_wait(bar_kv, 0, abort);
+            // S^T_i = K Q_i^T into region(i) (waits for the slice)
+            auto issue_st = [&](int i) -> bool {
+                const int st = i % QS;
+                if (!mbar_wait(bar_qf + st, (i / QS) & 1, abort)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                    umma_ss(tmem + region(i), sdesc_sw128(k_s + off, 16, 1024),
+                            sdesc_sw128(q_s + st * C::QT + off, 16, 1024), id_st, kk > 0);
+                }
+                umma_commit(bar_sf);
+                return true;
+            };
+            // dP^T_i = V dO_i^T into region(i + 1); the slice landed with Q_i
+            auto issue_dpt = [&](int i) {
+                const int st = i % QS;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+                    umma_ss(tmem + region(i + 1), sdesc_sw128(v_s + off, 16, 1024),
+                            sdesc_sw128(do_s + st * C::QT + off, 16, 1024), id_st, kk > 0);
+                }
+                umma_commit(bar_dpf);
+            };
+            // dV += P^T_i dO_i: P^T_i rows [32g, 32g + 32) packed into columns
+            // [32g, 32g + 16) of region(i)
+            auto issue_dv = [&](int i) -> bool {
+                const int st = i % QS;
+                if (!mbar_wait(bar_ptf, i & 1, abort)) return false;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BM / 16; ++kk)
+                    umma_ts(tmem + C::T_DV, tmem + region(i) + (kk >> 1) * 32 + (kk & 1) * 8,
+                            sdesc_sw128(do_s + st * C::QT + kk * 2048, BM * 128, 1024), id_acc,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+                return true;
+            };
+            // dK += dS^T_i Q_i (dS^T K-major) and dQ_i = dS_i K into region(i)
+            // (dS MN-major: the same tile; K MN-major), after dV_i read P^T_i there
+            auto issue_dk_dq = [&](int i) {
+                const int st = i % QS;
+#pragma unroll
+                for (int kk = 0; kk < BM / 16; ++kk)
+                    umma_ss(tmem + C::T_DK,
+                            sdesc_sw128(ds_s + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024),
+                            sdesc_sw128(q_s + st * C::QT + kk * 2048, BM * 128, 1024), id_acc,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bar_qe + st);  // Q_i and dO_i are no longer read
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_ss(tmem + region(i), sdesc_sw128(ds_s + kk * 2048, BN * 128, 1024),
+                            sdesc_sw128(k_s + kk * 2048, BN * 128, 1024), id_dq, kk > 0 ? 1u : 0u);
+                umma_commit(bar_dqf);
+            };
+            if (ok && nsteps > 0) {
+                ok = issue_st(0);
+                if (ok) issue_dpt(0);
+                for (int i = 0; ok && i < nsteps; ++i) {
+                    ok = issue_dv(i);
+                    if (ok) ok = mbar_wait(bar_dsf, i & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    // S^T_{i+1} overwrites dP^T_i, which the element-wise warps have read
+                    if (i + 1 < nsteps) ok = issue_st(i + 1);
+                    if (!ok) break;
+                    issue_dk_dq(i);
+                    if (i + 1 < nsteps) {
+                        ok = mbar_wait(bar_dqe, i & 1, abort);
+                        if (ok) {
+                            tc_fence_after();
+                            issue_dpt(i + 1);
+                        }
+                    }
+                }
+            }
+            umma_commit(bar_done);
+            drain_wait(bar_done, 0);
+        }
+    } else {
+        // ----------------------------------------------------- element-wise --
+        // S^T / dP^T: thread = (key = TMEM lane, quarter eg of a step's rows);
+        // dQ_i: thread = (row of the slice = TMEM lane, quarter eg of D)
+        const int quad = warp & 3;
+        const int eg = (warp - 2) >> 2;
+        const int sl = quad * 32 + lane;   // TMEM lane
+        const int s = ks + sl;             // local key index
+        const int tid = threadIdx.x - 64;  // 0 .. EW_THREADS-1
+        const float sl2 = P.scale * 1.4426950408889634f;
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        constexpr int HC = BM / EW;  // rows per thread and step
+        constexpr int DC = D / EW;   // dQ columns per thread
+        uint8_t *ds_tile = smem + C::OFF_DS;
+        float *r_lse = reinterpret_cast<float *>(smem + C::OFF_ROW);  // exp2 domain
+        float *r_d = r_lse + BM;
+        int *r_lo = reinterpret_cast<int *>(r_d + BM);
+        int *r_hi = r_lo + BM;
+        int *r_full = r_hi + BM;  // [0] largest lo, [1] smallest hi of the step
+        // Row data of a step (lse, D_t, the row's key interval, and the step's
+        // fully visible key range), gathered by threads 0..127 a step ahead.
+        struct RowData {
+            float L, dd;
+            int lo, hi, flo, fhi;
+        };
+        auto gather = [&](int i) -> RowData {
+            RowData d{-INFINITY, 0.f, 1, 0, 1, 0};
+            const int t0 = tbeg + i * BM;
+            const int t = t0 + tid;
+            if (tid < BM && i < nsteps && t <= tend && t < P.Tq) {
+                if (row_interval(P.mask, t, d.lo, d.hi) != 0) { d.lo = 1; d.hi = 0; }
+                d.L = __ldg(lse + ((int64_t)b * P.H + h) * P.Tq + t);
+                d.dd = __ldg(Dws + ((int64_t)b * P.H + h) * P.Tq + t);
+            }
+            if (tid == 0 && i < nsteps) {
+                // every row of the step valid: the interval ends are monotone, so the
+                // step is fully visible to keys in [lo(last row), hi(first row)]
+                const int tl_ = t0 + BM - 1;
+                int lo1 = 1, hi1 = 0, lo0 = 1, hi0 = 0;
+                if (tl_ <= tend && tl_ < P.Tq && row_interval(P.mask, tl_, lo1, hi1) == 0 &&
+                    row_interval(P.mask, t0, lo0, hi0) == 0) {
+                    d.flo = lo1;
+                    d.fhi = hi0;
+                }
+            }
+            return d;
+        };
+        // dQ_j: TMEM -> registers -> the dS^T tile (free once dQ_j is complete),
+        // one half slice (64 rows, the D / 32 swizzled boxes of tm_dq) at a time
+        // -> TMA reduce-add into the accumulator rows (b, h, tbeg + 128 j + r).
+        // Rows past the slice's end add zeros (their dS is 0); rows past the
+        // tensor's last row are clipped by the tensor map.
+        auto write_dq = [&](int j) -> bool {
+            if (!group_all(mbar_wait(bar_dqf, j & 1, abort))) return false;
+            tc_fence_after();
+            uint32_t a[DC];
+            tmem_ldn<DC>(tl + region(j) + eg * DC, a);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(bar_dqe);  // region(j) may take dP^T_{j+1}
+            const int row0 = (b * P.H + h) * P.Tq + tbeg + j * BM;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                if ((quad >> 1) == half) {
+                    const int rl = (quad & 1) * 32 + lane;  // row within the half slice
+#pragma unroll
+                    for (int c = 0; c < DC / 4; ++c) {
+                        const int col = eg * DC + 4 * c;
+                        const int ch = (col % DQ_BOX_COLS) / 4;
+                        uint8_t *dst = ds_tile + (col / DQ_BOX_COLS) * (DQ_BOX_ROWS * 128) +
+                                       rl * 128 + ((ch ^ (rl & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(dst) =
+                            make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
+                    }
+                    fence_proxy_async_smem();
+                }
+                ew_sync();  // the half slice is staged
+                if (tid == 0) {
+#pragma unroll
+                    for (int bx = 0; bx < D / DQ_BOX_COLS; ++bx)
+                        tma_reduce_add_2d(&tm_dq, ds_tile + bx * (DQ_BOX_ROWS * 128),
+                                          bx * DQ_BOX_COLS, row0 + half * DQ_BOX_ROWS);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                __syncwarp();
+                ew_sync();  // the staging has been read: the tile is free again
+            }
+            return true;
+        };
+        RowData next = gather(0);
+        bool ok = !skip;
+        for (int i = 0; i < nsteps; ++i) {
+            if (i > 0) ew_sync();  // every thread is done with step i-1's row data
+            if (ok && tid < BM) {
+                r_lse[tid] = (next.L == -INFINITY) ? INFINITY : next.L * 1.4426950408889634f;
+                r_d[tid] = next.dd;
+                r_lo[tid] = next.lo;
+                r_hi[tid] = next.hi;
+                if (tid == 0) {
+                    r_full[0] = next.flo;
+                    r_full[1] = next.fhi;
+                }
+            }
+            next = gather(i + 1);
+            ok = group_all(ok);  // row data written; all element-wise warps agree to go on
+            if (!ok) break;
+            // ---- P^T_i = exp(S^T_i scale - lse) over region(i)
+            ok = group_all(mbar_wait(bar_sf, i & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[HC];
+            tmem_ldn<HC>(tl + region(i) + eg * HC, v);
+            tmem_ld_wait();
+            const bool full = r_full[0] <= s && s <= r_full[1];
+            const float *cl = r_lse + eg * HC;
+            float p[HC];
+            if (full) {
+#pragma unroll
+                for (int r = 0; r < HC; ++r) p[r] = ex2(fmaf(__uint_as_float(v[r]), sl2, -cl[r]));
+            } else {
+                const int *clo = r_lo + eg * HC, *chi = r_hi + eg * HC;
+#pragma unroll
+                for (int r = 0; r < HC; ++r) {
+                    const bool vis = (clo[r] <= s) && (s <= chi[r]);
+                    p[r] = vis ? ex2(fmaf(__uint_as_float(v[r]), sl2, -cl[r])) : 0.f;
+                }
+            }
+            {
+                uint32_t pk[HC / 2];
+#pragma unroll
+                for (int c = 0; c < HC / 2; ++c) pk[c] = pack_bf16(p[2 * c], p[2 * c + 1]);
+                tmem_stn<HC / 2>(tl + region(i) + eg * HC, pk);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_ptf);
+            // ---- dQ_{i-1} out (its commit also covers dK_{i-1}: the tile is free)
+            if (i > 0) {
+                ok = write_dq(i - 1);
+                if (!ok) break;
+            }
+            // ---- dS^T_i = P^T_i (dP^T_i - D) into the shared tile
+            ok = group_all(mbar_wait(bar_dpf, i & 1, abort));
+            if (!ok) break;
+            tc_fence_after();
+            tmem_ldn<HC>(tl + region(i + 1) + eg * HC, v);
+            tmem_ld_wait();
+            const float *cd = r_d + eg * HC;
+#pragma unroll
+            for (int r = 0; r < HC; ++r) p[r] = p[r] * (__uint_as_float(v[r]) - cd[r]);
+            // key sl, rows [eg * HC, eg * HC + HC): 16-byte chunks eg * 4 .. eg * 4 + 3
+            // of the key's 256-byte row of the swizzled tile
+#pragma unroll
+            for (int j = 0; j < HC / 8; ++j) {
+                uint4 u;
+                u.x = pack_bf16(p[8 * j + 0], p[8 * j + 1]);
+                u.y = pack_bf16(p[8 * j + 2], p[8 * j + 3]);
+                u.z = pack_bf16(p[8 * j + 4], p[8 * j + 5]);
+                u.w = pack_bf16(p[8 * j + 6], p[8 * j + 7]);
+                *reinterpret_cast<uint4 *>(ds_tile + sw128_offset(sl, eg * (HC / 8) + j, BN)) = u;
+            }
+            tc_fence_before();        // dP^T_i read: region(i + 1) may take S^T_{i+1}
+            fence_proxy_async_smem();  // dS^T_i visible to the tensor pipe
+            mbar_arrive(bar_dsf);
+        }
+        if (ok && nsteps > 0) ok = write_dq(nsteps - 1);
+        if (tid == 0) bulk_wait_all();  // the last reduce-adds have landed
+        // ------------------------------------------------------ epilogue ---
+        // each warpgroup writes a quarter of the D columns of its keys' dV and dK
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort));
+        tc_fence_after();
+        constexpr int NCH = D / 16 / EW;  // 16-column chunks per warpgroup
+#pragma unroll 1
+        for (int q = 0; q < 2 * NCH; ++q) {  // dV chunks, then dK chunks
+            const int c = eg * NCH + (q % NCH);
+            const bool is_k = q >= NCH;
+            uint32_t a[16];
+            if (ok && nsteps > 0) {
+                tmem_ldn<16>(tl + (is_k ? C::T_DK : C::T_DV) + c * 16, a);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) a[e] = 0u;
+            }
+            if (ok && s < P.Tk) {
+                const int64_t off = b * P.kv_sb + (int64_t)s * P.kv_st + (int64_t)h * D + c * 16;
+                grad_out16(P, is_k ? dk : dv, off, reinterpret_cast<const float *>(a),
+                           is_k ? P.scale : 1.f);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace kvq
 }  // namespace tcbwd
 
 constexpr bool kTcBwdAvailable = true;

@@ -515,6 +515,20 @@ inline bool make_tmap_bf16(CUtensorMap *m, const void *base, int rank, const uin
     return r == CUDA_SUCCESS;
 }
 
+// 2-D tensor map over a row-major fp32 matrix [rows, cols] (row stride = cols);
+// box = box_cols x box_rows with the 128-byte swizzle (box_cols * 4 = 128).
+inline bool make_tmap_f32_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows,
+                             uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return false;
+    cuuint64_t gd[2] = {cols, rows}, gs[1] = {cols * 4};
+    cuuint32_t box[2] = {box_cols, box_rows}, es[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), gd, gs, box,
+                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Tensor maps of q-like [B, T, H, D] and cache-like [B, NB, T, H, D] operands.
 inline bool make_q_tmap(CUtensorMap *m, const void *base, const Problem &P, uint32_t box_rows) {
     const uint64_t dims[4] = {(uint64_t)P.D, (uint64_t)P.H, (uint64_t)P.Tq, (uint64_t)P.B};

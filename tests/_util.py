@@ -72,8 +72,8 @@ def gpu_fwd(inp, impl="auto", out_dtype=None):
                   causal=inp.get("causal", True), impl=impl, out_dtype=out_dtype)
 
 
-def gpu_bwd(inp, out, lse, impl="auto"):
+def gpu_bwd(inp, out, lse, impl="auto", deterministic=False):
     return ea.bwd(inp["grad_out"], inp["q"], inp["cache_k"], inp["cache_v"], out, lse,
                   inp["scale"], cu_seqlens=inp.get("cu_seqlens"), max_seqlen=inp.get("max_seqlen"),
                   q_pos_offset=inp.get("q_pos_offset", 0), k_pos_offset=inp.get("k_pos_offset", 0),
-                  causal=inp.get("causal", True), impl=impl)
+                  causal=inp.get("causal", True), impl=impl, deterministic=deterministic)

@@ -45,22 +45,31 @@ def test_chunked_bwd_matches_oracle_and_unchunked(T, H, D, NB, cp):
         assert max_abs(dv[:, :, :, h:h + 1], ov) <= TB["grad"]
 
 
-def test_grad_accumulate_adds_exactly():
-    """Accumulating twice into zeros gives exactly twice one accumulation, and
-    one accumulation rounds to the stored (bf16) gradient."""
+@pytest.mark.parametrize("deterministic", [True, False])
+def test_grad_accumulate_adds_exactly(deterministic):
+    """Accumulating twice into zeros gives twice one accumulation, and one
+    accumulation rounds to the stored (bf16) gradient: exactly with the
+    reproducible backward; with the default one, dk / dv exactly and dq (its
+    key tiles' contributions summed by fp32 atomics in varying order) to
+    within fp32 rounding and one bf16 ulp."""
     q, k, v, g = _inputs(640, 2, 128, 3, seed=5)
     out, lse = ea.fwd(q, k, v)
     bufs = [torch.zeros(q.shape, dtype=torch.float32, device="cuda"),
             torch.zeros(k.shape, dtype=torch.float32, device="cuda"),
             torch.zeros(k.shape, dtype=torch.float32, device="cuda")]
-    ea.bwd(g, q, k, v, out, lse, dq=bufs[0], dk=bufs[1], dv=bufs[2], grad_accumulate=True)
+    kw = dict(deterministic=deterministic)
+    ea.bwd(g, q, k, v, out, lse, dq=bufs[0], dk=bufs[1], dv=bufs[2], grad_accumulate=True, **kw)
     once = [b.clone() for b in bufs]
-    ea.bwd(g, q, k, v, out, lse, dq=bufs[0], dk=bufs[1], dv=bufs[2], grad_accumulate=True)
-    ref = ea.bwd(g, q, k, v, out, lse)
+    ea.bwd(g, q, k, v, out, lse, dq=bufs[0], dk=bufs[1], dv=bufs[2], grad_accumulate=True, **kw)
+    ref = ea.bwd(g, q, k, v, out, lse, **kw)
     torch.cuda.synchronize()
-    for b, o, r in zip(bufs, once, ref):
-        assert torch.equal(b, 2 * o)
-        assert torch.equal(o.to(torch.bfloat16), r)
+    for i, (b, o, r) in enumerate(zip(bufs, once, ref)):
+        if deterministic or i > 0:
+            assert torch.equal(b, 2 * o)
+            assert torch.equal(o.to(torch.bfloat16), r)
+        else:
+            assert max_abs(b, 2 * o) <= 1e-5
+            assert max_abs(o.to(torch.bfloat16), r) <= 2 ** -6
 
 
 @pytest.mark.slow
