@@ -306,18 +306,15 @@ def workload_config(w) -> dict:
 
 
 # ------------------------------------------------------------------ ours --
-def ours_arm(args, w, world, rank, local):
-    import online_softmax_merge_eagle_b200 as ea
-    from online_softmax_merge_eagle_b200.inputs import make_workload
+def make_step(args, w, ea, inp, inp_cpu, dev):
+    """Device buffers for workload w and a step(prof) closure that runs one
+    forward + backward through the library.  prof = dict of (start, stop)
+    torch.cuda.Event pairs: "fwd" and "bwd" bracket the main attention
+    kernels (the library records them on its launch stream), "bwd_all" the
+    whole backward call."""
     from online_softmax_merge_eagle_b200.schedules import (varlen_zigzag_backward,
                                                            varlen_zigzag_forward, zigzag_backward,
                                                            zigzag_forward)
-
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    pk = peaks()
-    inp_cpu = make_workload(w)
-    inp = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in inp_cpu.items()}
     cu = None if inp["cu_seqlens"] is None else torch.as_tensor(inp["cu_seqlens"], device=dev)
     kw = dict(cu_seqlens=cu, max_seqlen=inp["max_seqlen"], q_pos_offset=w.q_pos_offset,
               k_pos_offset=w.k_pos_offset, impl=args.kernel_impl)
@@ -331,81 +328,150 @@ def ours_arm(args, w, world, rank, local):
     ws = None
     if w.backward:
         ws = torch.empty(ea.bwd_workspace_size(q, k, v, **kw), dtype=torch.uint8, device=dev)
-    fl = flops(w)
+    det = bool(args.deterministic)
 
-    def step(prof_f=None, prof_b=None):
-        # NVTX range per step, visible to nsys / ncu --nvtx
-        torch.cuda.nvtx.range_push("eagle_step")
-        try:
-            step_body(prof_f, prof_b)
-        finally:
-            torch.cuda.nvtx.range_pop()
+    def rec(prof, key, i):
+        if prof is not None and key in prof:
+            prof[key][i].record()
 
-    def step_body(prof_f=None, prof_b=None):
+    def body(prof):
         if w.chunks and w.doc_lengths:
             # packed documents, each through the zig-zag chunk schedule
             cu_h = inp_cpu["cu_seqlens"]
-            if prof_f is not None:
-                prof_f[0].record()
+            rec(prof, "fwd", 0)
             varlen_zigzag_forward(q, k, v, w.scale, cu_h, cp=w.chunks // 2,
                                   impl=args.kernel_impl, out=out, lse=lse)
-            if prof_f is not None:
-                prof_f[1].record()
+            rec(prof, "fwd", 1)
             if w.backward:
-                if prof_b is not None:
-                    prof_b[0].record()
+                rec(prof, "bwd", 0)
                 varlen_zigzag_backward(g, q, k, v, out, lse, w.scale, cu_h, cp=w.chunks // 2,
-                                       impl=args.kernel_impl, dq=dq, dk=dk, dv=dv)
-                if prof_b is not None:
-                    prof_b[1].record()
+                                       impl=args.kernel_impl, dq=dq, dk=dk, dv=dv,
+                                       deterministic=det)
+                rec(prof, "bwd", 1)
             return
         if w.chunks:
             # block 0 through the zig-zag chunk schedule (emulated cp = chunks / 2)
-            if prof_f is not None:
-                prof_f[0].record()
+            rec(prof, "fwd", 0)
             zigzag_forward(q, k, v, w.scale, cp=w.chunks // 2, impl=args.kernel_impl, out=out,
                            lse=lse, single_launch=w.single_launch)
-            if prof_f is not None:
-                prof_f[1].record()
+            rec(prof, "fwd", 1)
             if w.backward:
-                if prof_b is not None:
-                    prof_b[0].record()
+                rec(prof, "bwd", 0)
                 zigzag_backward(g, q, k, v, out, lse, w.scale, cp=w.chunks // 2,
-                                impl=args.kernel_impl, dq=dq, dk=dk, dv=dv)
-                if prof_b is not None:
-                    prof_b[1].record()
+                                impl=args.kernel_impl, dq=dq, dk=dk, dv=dv, deterministic=det)
+                rec(prof, "bwd", 1)
             return
-        ea.fwd(q, k, v, w.scale, out=out, lse=lse, prof=prof_f, **kw)
+        ea.fwd(q, k, v, w.scale, out=out, lse=lse, prof=None if prof is None else prof["fwd"],
+               **kw)
         if w.backward:
-            ea.bwd(g, q, k, v, out, lse, w.scale, workspace=ws, dq=dq, dk=dk, dv=dv, prof=prof_b,
-                   **kw)
+            rec(prof, "bwd_all", 0)
+            ea.bwd(g, q, k, v, out, lse, w.scale, workspace=ws, dq=dq, dk=dk, dv=dv,
+                   prof=None if prof is None else prof["bwd"], deterministic=det, **kw)
+            rec(prof, "bwd_all", 1)
 
-    clocks = Clocks(local) if rank == 0 else None  # sampling starts before the warm-up
-    for _ in range(args.warmup):
+    def step(prof=None):
+        # NVTX range per step, visible to nsys / ncu --nvtx
+        torch.cuda.nvtx.range_push("eagle_step")
+        try:
+            body(prof)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    return step, kw, (q, k, v)
+
+
+def time_steps(step, steps, warmup, world, ea):
+    """W untimed steps, then exactly `steps` steps between a barrier and a
+    synchronize on both sides, timed with CUDA events on the launching stream.
+    Returns (ms per step, per-kernel mean ms, launches, wall window)."""
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    pf = [(ev(), ev()) for _ in range(args.steps)]
-    pb = [(ev(), ev()) for _ in range(args.steps)] if w.backward else [None] * args.steps
+    profs = [{key: (ev(), ev()) for key in ("fwd", "bwd", "bwd_all")} for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     n0 = ea.launch_count()
     t0, t1 = ev(), ev()
     wall0 = time.time()
     t0.record()
-    for i in range(args.steps):
-        step(pf[i], pb[i])
+    for i in range(steps):
+        step(profs[i])
     t1.record()
     torch.cuda.synchronize()
     wall1 = time.time()
     n1 = ea.launch_count()
     barrier(world)
+
+    def mean_ms(key):
+        vals = []
+        for pr in profs:
+            a, b = pr[key]
+            try:
+                vals.append(a.elapsed_time(b))
+            except RuntimeError:  # never recorded (e.g. no backward)
+                return 0.0
+        return statistics.mean(vals)
+    kern = {"fwd_ms": mean_ms("fwd"), "bwd_block0_ms": mean_ms("bwd"),
+            "bwd_all_ms": mean_ms("bwd_all")}
+    return t0.elapsed_time(t1) / steps, kern, n1 - n0, (wall0, wall1)
+
+
+def roofline_entry(achieved, peak, unit, bound, per_unit, units, peak_kind):
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": (achieved / peak) if achieved else None, "peak_kind": peak_kind,
+            "per_unit": per_unit, "units_per_launch": units}
+
+
+def kernel_rooflines(w, fl, kern, pk, det=False):
+    """Per-kernel entries: algorithmic work per launch / its mean CUDA-event
+    duration, against the measured burst bf16 peak (tensor kernels, timed in
+    a sub-second region) or the measured copy bandwidth (row pass)."""
+    burst = pk["bf16_tflops"]
+    src = " (" + pk["source"] + ")"
+    out = {}
+    if kern["fwd_ms"] > 0:
+        a = fl["fwd"] / (kern["fwd_ms"] * 1e-3) / 1e12
+        out["fwd"] = roofline_entry(a, burst, "TFLOP/s", "tensor",
+                                    "4*D FLOP per pair + 4*D per row and diagonal block",
+                                    fl["pairs"], "bf16_tflops burst" + src)
+    if w.backward and kern["bwd_block0_ms"] > 0:
+        a = 10 * w.D * fl["pairs"] / (kern["bwd_block0_ms"] * 1e-3) / 1e12
+        out["bwd_block0"] = roofline_entry(a, burst, "TFLOP/s", "tensor", "10*D FLOP per pair",
+                                           fl["pairs"], "bf16_tflops burst" + src)
+    if w.backward and kern["bwd_all_ms"] > kern["bwd_block0_ms"] > 0 and not w.chunks:
+        rows = w.B * w.Tq * w.H
+        es = 2  # bf16
+        per_row = (3 * w.D * es + (w.num_blocks - 1) * 4 * w.D * es + 8
+                   + (4 * w.D if w.num_blocks > 1 or not det else 0))
+        ms = kern["bwd_all_ms"] - kern["bwd_block0_ms"]
+        gbs = rows * per_row / (ms * 1e-3) / 1e9
+        e = roofline_entry(gbs, pk["hbm_gbs"], "GB/s", "hbm",
+                           "bytes per row: dO, O, q + (NB-1) x (k, v read, dk, dv write) "
+                           "+ the fp32 dQ accumulator row written + lse, D_t", rows,
+                           "hbm_gbs" + src)
+        e["kernel"] = "bwd_rows_kernel (bwd call minus its block-0 kernels)"
+        out["bwd_rows"] = e
+    return out
+
+
+def ours_arm(args, w, world, rank, local):
+    import online_softmax_merge_eagle_b200 as ea
+    from online_softmax_merge_eagle_b200.inputs import WORKLOADS, make_workload
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    inp_cpu = make_workload(w)
+    inp = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in inp_cpu.items()}
+    step, kw, (q, k, v) = make_step(args, w, ea, inp, inp_cpu, dev)
+    fl = flops(w)
+
+    clocks = Clocks(local) if rank == 0 else None  # sampling starts before the warm-up
+    ms, kern, launches, (wall0, wall1) = time_steps(step, args.steps, args.warmup, world, ea)
     clk = clocks.stop(wall0, wall1) if clocks else None
-    ms = t0.elapsed_time(t1)
-    ms_step = max_over_ranks(ms / args.steps, world, dev)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in pf)
-    bwd_ms = statistics.mean(a.elapsed_time(b) for a, b in pb) if w.backward else 0.0
-    launches = (n1 - n0) // 1
+    ms_step = max_over_ranks(ms, world, dev)
+    fwd_ms, bwd_ms = kern["fwd_ms"], kern["bwd_block0_ms"]
 
     tflops = job_tflops(world, fl["total"], ms_step)
     tokens = world * w.B * w.Tq / (ms_step * 1e-3)
@@ -416,10 +482,40 @@ def ours_arm(args, w, world, rank, local):
         dom, achieved = "bwd_block0", bwd_main_tf
     else:
         dom, achieved = "fwd", fwd_main_tf
-    peak = pk["bf16_tflops_sustained"]
+    # the timed region is well under a second: the burst cuBLAS figure applies
+    peak = pk["bf16_tflops"]
+    per_kernel = kernel_rooflines(w, fl, kern, pk, bool(args.deterministic))
 
     e2e = e2e_measure(args, w, inp_cpu, kw, ea, dev, fl, world) if not args.no_e2e else None
     merge = merge_measure(ea, dev, pk) if not args.no_merge else None
+    if merge:
+        per_kernel["merge"] = roofline_entry(merge["GBps"], pk["hbm_gbs"], "GB/s", "hbm",
+                                             "D*(4+4+2)+12 bytes per row (bf16 block)",
+                                             merge["bytes_per_launch"] // (128 * 10 + 12),
+                                             "hbm_gbs (" + pk["source"] + ")")
+    del inp, step
+    extra = {}
+    for name in ([] if args.no_extra else [x for x in args.extra.split(",") if x]):
+        if name == w.name:
+            continue
+        xw = WORKLOADS[name]
+        xcpu = make_workload(xw)
+        xin = {n: (x.to(dev) if isinstance(x, torch.Tensor) else x) for n, x in xcpu.items()}
+        xstep, _, _ = make_step(args, xw, ea, xin, xcpu, dev)
+        xfl = flops(xw)
+        xms, xkern, _, _ = time_steps(xstep, max(3, args.steps // 2), args.warmup, world, ea)
+        xms = max_over_ranks(xms, world, dev)
+        extra[name] = {"value": job_tflops(world, xfl["total"], xms), "unit": "TFLOP/s",
+                       "ms_per_step": xms, "flop_per_step": xfl,
+                       "kernels": {**xkern,
+                                   "fwd_tflops": xfl["fwd"] / (xkern["fwd_ms"] * 1e-3) / 1e12
+                                   if xkern["fwd_ms"] > 0 else None,
+                                   "bwd_block0_tflops": 10 * xw.D * xfl["pairs"] /
+                                   (xkern["bwd_block0_ms"] * 1e-3) / 1e12
+                                   if xkern["bwd_block0_ms"] > 0 else None},
+                       "roofline": kernel_rooflines(xw, xfl, xkern, pk, bool(args.deterministic)),
+                       "steps": max(3, args.steps // 2), "warmup": args.warmup}
+        del xin, xstep
 
     if rank != 0:
         return 0
@@ -437,6 +533,7 @@ def ours_arm(args, w, world, rank, local):
     cfg["l2"] = "inputs larger than L2 (%.2f GB read per step)" % (
         sum(t.numel() * t.element_size() for t in (q, k, v)) / 1e9)
     cfg["parallelism"] = f"replica x{world}"
+    cfg["deterministic_bwd"] = bool(args.deterministic)
     line = {
         "metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -449,16 +546,22 @@ def ours_arm(args, w, world, rank, local):
                           "of_nominal_2250": tflops / world / 2250.0},
         "flop_per_step": fl,
         "kernels": {"fwd_ms": fwd_ms, "fwd_tflops": fwd_main_tf, "bwd_block0_ms": bwd_ms,
-                    "bwd_block0_tflops": bwd_main_tf, "impl": args.kernel_impl},
+                    "bwd_block0_tflops": bwd_main_tf, "bwd_all_ms": kern["bwd_all_ms"],
+                    "impl": args.kernel_impl,
+                    "bwd_mode": "deterministic pair" if args.deterministic else
+                    "five products per tile pair (dQ by TMA reduce-add)"},
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": (achieved / peak) if achieved else None,
-                     "peak_kind": "bf16_tflops_sustained (" + pk["source"] + ")",
-                     "frac_of_burst": (achieved / pk["bf16_tflops"]) if achieved else None,
+                     "peak_kind": "bf16_tflops burst (" + pk["source"] + ")",
+                     "frac_of_sustained": (achieved / pk["bf16_tflops_sustained"])
+                     if achieved else None,
                      "traffic": dram_traffic(w.name, dom),
                      "traffic_source": TRAFFIC_FILE},
+        "roofline_per_kernel": per_kernel,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "merge": merge,
+        "extra_workloads": extra or None,
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -525,7 +628,8 @@ def e2e_measure(args, w, inp, kw, ea, dev, fl, world):
             ea.fwd(d["q"], d["cache_k"], d["cache_v"], w.scale, out=o["out"], lse=o["lse"], **kw)
             if w.backward:
                 ea.bwd(d["grad_out"], d["q"], d["cache_k"], d["cache_v"], o["out"], o["lse"],
-                       w.scale, workspace=ws, dq=o["dq"], dk=o["dk"], dv=o["dv"], **kw)
+                       w.scale, workspace=ws, dq=o["dq"], dk=o["dk"], dv=o["dv"],
+                       deterministic=bool(args.deterministic), **kw)
         ev = torch.cuda.Event()
         ev.record(compute)
         return ev
@@ -616,6 +720,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-merge", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deterministic", type=int, default=0,
+                    help="1: the reproducible backward pair instead of the five-product kernel")
+    ap.add_argument("--extra", default="varlen_bf16",
+                    help="comma-separated workloads also timed (device only) in the same run")
+    ap.add_argument("--no-extra", action="store_true")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     w = WORKLOADS[args.workload]

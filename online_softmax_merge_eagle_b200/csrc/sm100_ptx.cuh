@@ -288,6 +288,14 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Adds four fp32 values to 16 bytes of global memory (one vector reduction,
+// no return value; the address must be 16-byte aligned).
+__device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);

@@ -728,48 +728,63 @@ __global__ void __launch_bounds__(THREADS, 1)
 // to the fp32 dQ accumulator in global memory (the order of those fp32
 // additions across CTAs varies from run to run).  dS^T goes to shared memory
 // once, bf16 with the 128-byte swizzle, and serves as the K-major A operand of
-// dK += dS^T Q and as the MN-major A operand of dQ_i = dS K.  dQ_i leaves
-// through the same shared tile once both products have read it: two halves of
-// 64 rows, staged in the swizzled boxes of a TMA tensor map over the
-// accumulator and added there by TMA reduce-adds (whole L2 lines, a handful
-// of requests per slice instead of one per 16 bytes and thread).
+// dK += dS^T Q and as the MN-major A operand of dQ_i = dS K.
+// Shared memory: K, V, a ring of three Q slots and two dO slots; at D = 128
+// dS^T_i is written over dO_i once dV_i has read it (at D = 64 it has a tile
+// of its own).  dQ_i leaves through the slots of Q_i and dO_i, which no
+// product reads once dQ_i is complete: the element-wise warps stage it there
+// (fp32, in the swizzled boxes of a TMA tensor map over the accumulator), and
+// the producer warp, which owns the slots, issues TMA reduce-adds (whole L2
+// lines), waits until they have read the slots and then loads dO_{i+2} and
+// Q_{i+3} into them -- a step and two steps before they are needed, so the
+// reductions drain while the next steps compute.
 // TMEM: dV [0, D), dK [128, 128 + D) and two 128-column regions R0, R1 that
 // carry in turn S^T_i -> P^T_i (R_{i%2}), dP^T_i (R_{(i+1)%2}) and dQ_i
 // (R_{i%2}, issued after dV_i has read P^T_i).
 // MMA issue order: S^T_0, dP^T_0, then per step i: dV_i (once P^T_i is
 // written); S^T_{i+1}, dK_i, dQ_i (once dS^T_i is in shared memory);
 // dP^T_{i+1} (once the element-wise warps have read dQ_i out of R_{i%2}).
-// Element-wise order per step: P^T_i, then dQ_{i-1} out to global memory,
-// then dS^T_i.  Every wait of the element-wise warps is ANDed over all of
-// them (a named barrier), so they take every exit decision together.
+// Element-wise order per step: P^T_i, then dQ_{i-1} out, then dS^T_i.
 namespace kvq {
 
 constexpr int BN = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dV, dK)
 constexpr int BM = 128;  // query rows per step (TMEM lanes of dQ_i)
-constexpr int QS = 2;    // Q / dO ring depth
+constexpr int QSL = 3;   // Q slots
+constexpr int OSL = 2;   // dO slots
 constexpr int DQ_BOX_COLS = 32;  // fp32 box of the dQ tensor map: 32 columns (128 bytes)
-constexpr int DQ_BOX_ROWS = 64;  // x 64 rows (half a slice)
+constexpr int DQ_BOX_ROWS = BM;  // x the 128 rows of a slice
 
 template <int D>
 struct Cfg {
     static constexpr int KT = BN * D * 2;    // K or V tile bytes
-    static constexpr int QT = BM * D * 2;    // Q or dO slice bytes
-    static constexpr int DST = BN * BM * 2;  // dS^T tile bytes (also the dQ staging)
-    static_assert(DQ_BOX_ROWS * D * 4 <= DST, "a half dQ slice fits the dS^T tile");
+    static constexpr int QT = BM * D * 2;    // Q or dO slice bytes (one slot)
+    static constexpr int DST = BN * BM * 2;  // dS^T tile bytes
+    static constexpr bool DS_IN_DO = QT >= DST;  // dS^T_i over dO_i (D = 128)
+    static constexpr int BOX = DQ_BOX_ROWS * DQ_BOX_COLS * 4;  // one staged dQ box
+    static constexpr int NBOX = D / DQ_BOX_COLS;                // boxes per slice
+    static_assert((NBOX / 2) * BOX == QT, "half the dQ boxes fill a Q (or dO) slot");
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + KT;
     static constexpr int OFF_Q = OFF_V + KT;
-    static constexpr int OFF_DO = OFF_Q + QS * QT;
-    static constexpr int OFF_DS = OFF_DO + QS * QT;
-    static constexpr int OFF_ROW = OFF_DS + DST;  // lse2[BM], D[BM], lo[BM], hi[BM], 2 ints
+    static constexpr int OFF_DO = OFF_Q + QSL * QT;
+    static constexpr int OFF_DS = OFF_DO + OSL * QT;  // own dS^T tile (D = 64 only)
+    static constexpr int OFF_ROW = OFF_DS + (DS_IN_DO ? 0 : DST);  // lse2, D, lo, hi, 2 ints
     static constexpr int ROW_BYTES = 4 * BM * 4 + 16;
     static constexpr int OFF_BAR = OFF_ROW + ROW_BYTES;
-    static constexpr int NBARS = 12;  // >= the barriers laid out in the kernel
+    static constexpr int NBARS = 20;  // >= the barriers laid out in the kernel
     // no realignment slack: the kernel checks that the base is 1024-byte aligned
     static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16;
     static_assert(SMEM <= 232448, "shared memory");
     static constexpr uint32_t T_DV = 0, T_DK = 128, T_R0 = 256, T_R1 = 384, TMEM_COLS = 512;
     static_assert(D <= 128, "TMEM budget");
+    static __device__ __forceinline__ int q_off(int i) { return OFF_Q + (i % QSL) * QT; }
+    static __device__ __forceinline__ int do_off(int i) { return OFF_DO + (i % OSL) * QT; }
+    static __device__ __forceinline__ int ds_off(int i) { return DS_IN_DO ? do_off(i) : OFF_DS; }
+    // staged dQ box bx of slice i: the first half of the boxes over Q_i's slot,
+    // the second half over dO_i's
+    static __device__ __forceinline__ int box_off(int i, int bx) {
+        return (bx < NBOX / 2 ? q_off(i) : do_off(i)) + (bx % (NBOX / 2)) * BOX;
+    }
 };
 
 // Named barrier 2 over the element-wise warps.
@@ -795,15 +810,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     uint64_t *bars = (uint64_t *)(smem + C::OFF_BAR);
     uint64_t *bar_kv = bars + 0;
-    uint64_t *bar_qf = bars + 1, *bar_qe = bars + 1 + QS;  // QS each
-    uint64_t *bar_sf = bars + 1 + 2 * QS;  // S^T_i in TMEM
+    uint64_t *bar_qf = bars + 1;           // [QSL]: Q_i landed
+    uint64_t *bar_of = bar_qf + QSL;       // [OSL]: dO_i landed
+    uint64_t *bar_sf = bar_of + OSL;       // S^T_i in TMEM
     uint64_t *bar_dpf = bar_sf + 1;        // dP^T_i in TMEM
-    uint64_t *bar_dqf = bar_dpf + 1;       // dQ_i in TMEM (dK_i done too: dS^T free)
+    uint64_t *bar_dvd = bar_dpf + 1;       // dV_i done: dO_i no longer read
+    uint64_t *bar_dqf = bar_dvd + 1;       // dQ_i in TMEM (dK_i done too: dS^T free)
     uint64_t *bar_ptf = bar_dqf + 1;       // P^T_i written over S^T_i (EW_THREADS)
     uint64_t *bar_dsf = bar_ptf + 1;       // dS^T_i in shared memory, dP^T_i read (EW_THREADS)
     uint64_t *bar_dqe = bar_dsf + 1;       // dQ_i read out of TMEM (EW_THREADS)
-    uint64_t *bar_done = bar_dqe + 1;
-    static_assert(C::NBARS >= 1 + 2 * QS + 7, "barrier slots");
+    uint64_t *bar_stg = bar_dqe + 1;       // dQ_i staged over Q_i and dO_i (EW_THREADS)
+    uint64_t *bar_done = bar_stg + 1;
+    static_assert(C::NBARS >= 1 + QSL + OSL + 10, "barrier slots");
     uint32_t *tmem_slot = (uint32_t *)(bars + C::NBARS);
     volatile int *abort = (volatile int *)(tmem_slot + 1);
 
@@ -818,6 +836,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(bar_ptf, EW_THREADS);
         mbar_init(bar_dsf, EW_THREADS);
         mbar_init(bar_dqe, EW_THREADS);
+        mbar_init(bar_stg, EW_THREADS);
         *abort = status_bad() ? 1 : 0;
         fence_mbar_init();
     }
@@ -835,36 +854,56 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ producer --
+        // K, V, Q_0..Q_2 and dO_0, dO_1 first; then per step i: once dQ_i is
+        // staged over the slots of Q_i and dO_i, its reduce-adds into the
+        // accumulator rows (b, h, tbeg + 128 i + r) -- rows past the slice's end
+        // add zeros (their dS is 0), rows past the tensor's last row are clipped
+        // by the tensor map -- and, once they have read the slots, dO_{i+2} and
+        // Q_{i+3} into them
         if (lane == 0 && !skip) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_do);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_dq);
             mbar_expect_tx(bar_kv, 2 * C::KT);
 #pragma unroll
             for (int cb = 0; cb < D / 64; ++cb) {
                 tma_load_5d(smem + C::OFF_K + cb * BN * 128, &tm_k, bar_kv, cb * 64, h, ks, 0, b);
                 tma_load_5d(smem + C::OFF_V + cb * BN * 128, &tm_v, bar_kv, cb * 64, h, ks, 0, b);
             }
-            int issued = 0;
-            for (int i = 0; i < nsteps; ++i) {
-                const int st = i % QS;
-                const int t0 = tbeg + i * BM;
-                if (!mbar_wait(bar_qe + st, ((i / QS) & 1) ^ 1, abort)) break;
-                mbar_expect_tx(bar_qf + st, 2 * C::QT);
+            auto load = [&](bool is_do, int i) {
+                uint64_t *bar = is_do ? bar_of + i % OSL : bar_qf + i % QSL;
+                uint8_t *dst = smem + (is_do ? C::do_off(i) : C::q_off(i));
+                mbar_expect_tx(bar, C::QT);
 #pragma unroll
-                for (int cb = 0; cb < D / 64; ++cb) {
-                    tma_load_4d(smem + C::OFF_Q + st * C::QT + cb * BM * 128, &tm_q, bar_qf + st,
-                                cb * 64, h, t0, b);
-                    tma_load_4d(smem + C::OFF_DO + st * C::QT + cb * BM * 128, &tm_do, bar_qf + st,
-                                cb * 64, h, t0, b);
+                for (int cb = 0; cb < D / 64; ++cb)
+                    tma_load_4d(dst + cb * BM * 128, is_do ? &tm_do : &tm_q, bar, cb * 64, h,
+                                tbeg + i * BM, b);
+            };
+            int q_issued = 0, o_issued = 0;
+            for (; q_issued < QSL && q_issued < nsteps; ++q_issued) load(false, q_issued);
+            for (; o_issued < OSL && o_issued < nsteps; ++o_issued) load(true, o_issued);
+            for (int i = 0; i < nsteps; ++i) {
+                if (!mbar_wait(bar_stg, i & 1, abort)) break;
+                const int row0 = (b * P.H + h) * P.Tq + tbeg + i * BM;
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_reduce_add_2d(&tm_dq, smem + C::box_off(i, bx), bx * DQ_BOX_COLS, row0);
+                bulk_commit();
+                if (i + OSL < nsteps || i + QSL < nsteps) {
+                    bulk_wait_read_all();  // the slots are free again
+                    if (i + OSL < nsteps) load(true, o_issued++);
+                    if (i + QSL < nsteps) load(false, q_issued++);
                 }
-                issued = i + 1;
             }
+            bulk_wait_all();  // every reduce-add has landed
             if (*abort) {
                 drain_wait(bar_kv, 0);
-                for (int i = (issued > QS ? issued - QS : 0); i < issued; ++i)
-                    drain_wait(bar_qf + i % QS, (i / QS) & 1);
+                for (int i = (q_issued > QSL ? q_issued - QSL : 0); i < q_issued; ++i)
+                    drain_wait(bar_qf + i % QSL, (i / QSL) & 1);
+                for (int i = (o_issued > OSL ? o_issued - OSL : 0); i < o_issued; ++i)
+                    drain_wait(bar_of + i % OSL, (i / OSL) & 1);
             }
         }
     } else if (warp == 1) {
@@ -873,59 +912,61 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t id_st = idesc_bf16(BN, BM, false);      // M = 128 keys, N = 128 rows
             const uint32_t id_acc = idesc_bf16(BN, D, true);       // M = 128 keys, N = D, B MN-major
             const uint32_t id_dq = idesc_bf16(BM, D, true, true);  // M = 128 rows, N = D, A, B MN-major
-            const uint32_t k_s = smem_u32(smem + C::OFF_K), v_s = smem_u32(smem + C::OFF_V);
-            const uint32_t q_s = smem_u32(smem + C::OFF_Q), do_s = smem_u32(smem + C::OFF_DO);
-            const uint32_t ds_s = smem_u32(smem + C::OFF_DS);
+            const uint32_t base = smem_u32(smem);
+            const uint32_t k_s = base + C::OFF_K, v_s = base + C::OFF_V;
             bool ok = mbar_wait(bar_kv, 0, abort);
-            // S^T_i = K Q_i^T into region(i) (waits for the slice)
+            // S^T_i = K Q_i^T into region(i) (waits for Q_i)
             auto issue_st = [&](int i) -> bool {
-                const int st = i % QS;
-                if (!mbar_wait(bar_qf + st, (i / QS) & 1, abort)) return false;
+                if (!mbar_wait(bar_qf + i % QSL, (i / QSL) & 1, abort)) return false;
                 tc_fence_after();
+                const uint32_t q_s = base + C::q_off(i);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
                     umma_ss(tmem + region(i), sdesc_sw128(k_s + off, 16, 1024),
-                            sdesc_sw128(q_s + st * C::QT + off, 16, 1024), id_st, kk > 0);
+                            sdesc_sw128(q_s + off, 16, 1024), id_st, kk > 0);
                 }
                 umma_commit(bar_sf);
                 return true;
             };
-            // dP^T_i = V dO_i^T into region(i + 1); the slice landed with Q_i
-            auto issue_dpt = [&](int i) {
-                const int st = i % QS;
+            // dP^T_i = V dO_i^T into region(i + 1) (waits for dO_i)
+            auto issue_dpt = [&](int i) -> bool {
+                if (!mbar_wait(bar_of + i % OSL, (i / OSL) & 1, abort)) return false;
+                tc_fence_after();
+                const uint32_t do_s = base + C::do_off(i);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
                     umma_ss(tmem + region(i + 1), sdesc_sw128(v_s + off, 16, 1024),
-                            sdesc_sw128(do_s + st * C::QT + off, 16, 1024), id_st, kk > 0);
+                            sdesc_sw128(do_s + off, 16, 1024), id_st, kk > 0);
                 }
                 umma_commit(bar_dpf);
+                return true;
             };
             // dV += P^T_i dO_i: P^T_i rows [32g, 32g + 32) packed into columns
             // [32g, 32g + 16) of region(i)
             auto issue_dv = [&](int i) -> bool {
-                const int st = i % QS;
                 if (!mbar_wait(bar_ptf, i & 1, abort)) return false;
                 tc_fence_after();
+                const uint32_t do_s = base + C::do_off(i);
 #pragma unroll
                 for (int kk = 0; kk < BM / 16; ++kk)
                     umma_ts(tmem + C::T_DV, tmem + region(i) + (kk >> 1) * 32 + (kk & 1) * 8,
-                            sdesc_sw128(do_s + st * C::QT + kk * 2048, BM * 128, 1024), id_acc,
+                            sdesc_sw128(do_s + kk * 2048, BM * 128, 1024), id_acc,
                             (i > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bar_dvd);
                 return true;
             };
             // dK += dS^T_i Q_i (dS^T K-major) and dQ_i = dS_i K into region(i)
             // (dS MN-major: the same tile; K MN-major), after dV_i read P^T_i there
             auto issue_dk_dq = [&](int i) {
-                const int st = i % QS;
+                const uint32_t q_s = base + C::q_off(i), ds_s = base + C::ds_off(i);
 #pragma unroll
                 for (int kk = 0; kk < BM / 16; ++kk)
                     umma_ss(tmem + C::T_DK,
                             sdesc_sw128(ds_s + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024),
-                            sdesc_sw128(q_s + st * C::QT + kk * 2048, BM * 128, 1024), id_acc,
+                            sdesc_sw128(q_s + kk * 2048, BM * 128, 1024), id_acc,
                             (i > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(bar_qe + st);  // Q_i and dO_i are no longer read
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
                     umma_ss(tmem + region(i), sdesc_sw128(ds_s + kk * 2048, BN * 128, 1024),
@@ -934,7 +975,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             };
             if (ok && nsteps > 0) {
                 ok = issue_st(0);
-                if (ok) issue_dpt(0);
+                if (ok) ok = issue_dpt(0);
                 for (int i = 0; ok && i < nsteps; ++i) {
                     ok = issue_dv(i);
                     if (ok) ok = mbar_wait(bar_dsf, i & 1, abort);
@@ -946,10 +987,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     issue_dk_dq(i);
                     if (i + 1 < nsteps) {
                         ok = mbar_wait(bar_dqe, i & 1, abort);
-                        if (ok) {
-                            tc_fence_after();
-                            issue_dpt(i + 1);
-                        }
+                        if (ok) ok = issue_dpt(i + 1);
                     }
                 }
             }
@@ -969,7 +1007,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         constexpr int HC = BM / EW;  // rows per thread and step
         constexpr int DC = D / EW;   // dQ columns per thread
-        uint8_t *ds_tile = smem + C::OFF_DS;
         float *r_lse = reinterpret_cast<float *>(smem + C::OFF_ROW);  // exp2 domain
         float *r_d = r_lse + BM;
         int *r_lo = reinterpret_cast<int *>(r_d + BM);
@@ -1003,47 +1040,28 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             return d;
         };
-        // dQ_j: TMEM -> registers -> the dS^T tile (free once dQ_j is complete),
-        // one half slice (64 rows, the D / 32 swizzled boxes of tm_dq) at a time
-        // -> TMA reduce-add into the accumulator rows (b, h, tbeg + 128 j + r).
-        // Rows past the slice's end add zeros (their dS is 0); rows past the
-        // tensor's last row are clipped by the tensor map.
+        // dQ_j: TMEM -> registers -> the swizzled boxes of tm_dq over the slots
+        // of Q_j and dO_j (no product reads them once dQ_j is complete); the
+        // producer adds them into the accumulator
         auto write_dq = [&](int j) -> bool {
-            if (!group_all(mbar_wait(bar_dqf, j & 1, abort))) return false;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_dqf, j & 1, abort))) return false;
             tc_fence_after();
             uint32_t a[DC];
             tmem_ldn<DC>(tl + region(j) + eg * DC, a);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(bar_dqe);  // region(j) may take dP^T_{j+1}
-            const int row0 = (b * P.H + h) * P.Tq + tbeg + j * BM;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                if ((quad >> 1) == half) {
-                    const int rl = (quad & 1) * 32 + lane;  // row within the half slice
 #pragma unroll
-                    for (int c = 0; c < DC / 4; ++c) {
-                        const int col = eg * DC + 4 * c;
-                        const int ch = (col % DQ_BOX_COLS) / 4;
-                        uint8_t *dst = ds_tile + (col / DQ_BOX_COLS) * (DQ_BOX_ROWS * 128) +
-                                       rl * 128 + ((ch ^ (rl & 7)) << 4);
-                        *reinterpret_cast<uint4 *>(dst) =
-                            make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
-                    }
-                    fence_proxy_async_smem();
-                }
-                ew_sync();  // the half slice is staged
-                if (tid == 0) {
-#pragma unroll
-                    for (int bx = 0; bx < D / DQ_BOX_COLS; ++bx)
-                        tma_reduce_add_2d(&tm_dq, ds_tile + bx * (DQ_BOX_ROWS * 128),
-                                          bx * DQ_BOX_COLS, row0 + half * DQ_BOX_ROWS);
-                    bulk_commit();
-                    bulk_wait_read_all();
-                }
-                __syncwarp();
-                ew_sync();  // the staging has been read: the tile is free again
+            for (int c = 0; c < DC / 4; ++c) {
+                const int col = eg * DC + 4 * c;
+                const int ch = (col % DQ_BOX_COLS) / 4;
+                uint8_t *dst = smem + C::box_off(j, col / DQ_BOX_COLS) + sl * 128 +
+                               ((ch ^ (sl & 7)) << 4);
+                *reinterpret_cast<uint4 *>(dst) =
+                    make_uint4(a[4 * c], a[4 * c + 1], a[4 * c + 2], a[4 * c + 3]);
             }
+            fence_proxy_async_smem();  // visible to the TMA unit
+            mbar_arrive(bar_stg);
             return true;
         };
         RowData next = gather(0);
@@ -1061,11 +1079,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             next = gather(i + 1);
-            ok = group_all(ok);  // row data written; all element-wise warps agree to go on
+            // row data written; all element-wise warps agree to go on.  A warp whose
+            // wait fails below skips to the next iteration, where every warp stops
+            // here (the named barriers of an iteration all sit before its waits).
+            ok = group_all(ok);
             if (!ok) break;
             // ---- P^T_i = exp(S^T_i scale - lse) over region(i)
-            ok = group_all(mbar_wait(bar_sf, i & 1, abort));
-            if (!ok) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_sf, i & 1, abort));
+            if (!ok) continue;
             tc_fence_after();
             uint32_t v[HC];
             tmem_ldn<HC>(tl + region(i) + eg * HC, v);
@@ -1093,20 +1114,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             tc_fence_before();
             mbar_arrive(bar_ptf);
-            // ---- dQ_{i-1} out (its commit also covers dK_{i-1}: the tile is free)
+            // ---- dQ_{i-1} out
             if (i > 0) {
                 ok = write_dq(i - 1);
-                if (!ok) break;
+                if (!ok) continue;
             }
             // ---- dS^T_i = P^T_i (dP^T_i - D) into the shared tile
-            ok = group_all(mbar_wait(bar_dpf, i & 1, abort));
-            if (!ok) break;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_dpf, i & 1, abort));
+            if (!ok) continue;
             tc_fence_after();
             tmem_ldn<HC>(tl + region(i + 1) + eg * HC, v);
             tmem_ld_wait();
             const float *cd = r_d + eg * HC;
 #pragma unroll
             for (int r = 0; r < HC; ++r) p[r] = p[r] * (__uint_as_float(v[r]) - cd[r]);
+            // at D = 128 the tile is dO_i's slot: dV_i must have read it
+            if (C::DS_IN_DO) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_dvd, i & 1, abort));
+                if (!ok) continue;
+            }
+            uint8_t *ds_tile = smem + C::ds_off(i);
             // key sl, rows [eg * HC, eg * HC + HC): 16-byte chunks eg * 4 .. eg * 4 + 3
             // of the key's 256-byte row of the swizzled tile
 #pragma unroll
@@ -1123,7 +1150,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_arrive(bar_dsf);
         }
         if (ok && nsteps > 0) ok = write_dq(nsteps - 1);
-        if (tid == 0) bulk_wait_all();  // the last reduce-adds have landed
         // ------------------------------------------------------ epilogue ---
         // each warpgroup writes a quarter of the D columns of its keys' dV and dK
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_done, 0, abort));

@@ -114,7 +114,7 @@ def _chunk_schedule_forward(q, cache_k, cache_v, scale, n_chunks, rank_chunks, i
 
 
 def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, impl: str = "auto",
-                    dq=None, dk=None, dv=None, ranks=None, acc32=None):
+                    dq=None, dk=None, dv=None, ranks=None, acc32=None, deterministic=False):
     """Backward of the whole sequence through the zig-zag chunk schedule.
 
     Shapes as zigzag_forward; out / lse are the merged forward results of the
@@ -126,7 +126,8 @@ def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, imp
     contributions of the listed ranks are included.  ``acc32`` = (dq32, dk32,
     dv32): zeroed fp32 accumulators with q's / cache_k's element strides to use
     instead of fresh ones (the varlen schedule passes views of whole-sequence
-    buffers).
+    buffers).  ``deterministic`` selects the reproducible backward for every
+    pair (eagle_attn_params.deterministic).
     """
     B, T, H, D = q.shape
     if B != 1 or T % (2 * cp):
@@ -156,7 +157,8 @@ def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, imp
                     dkk, dvv = dk32[:, :, qs], dv32[:, :, qs]
                 bwd(grad_out[:, qs], q[:, qs], kk, vv, out[:, qs], lse_c, scale,
                     q_pos_offset=qc * c, k_pos_offset=kc * c, impl=impl, workspace=ws,
-                    dq=dq32[:, qs], dk=dkk, dv=dvv, grad_accumulate=True)
+                    dq=dq32[:, qs], dk=dkk, dv=dvv, grad_accumulate=True,
+                    deterministic=deterministic)
     dq = finalize(dq32, q.dtype, out=dq)
     if dk is None:
         dk = torch.empty_like(cache_k)
@@ -200,7 +202,7 @@ def varlen_zigzag_forward(q, cache_k, cache_v, scale, cu_seqlens, cp: int, impl:
 
 
 def varlen_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cu_seqlens, cp: int,
-                           impl: str = "auto", dq=None, dk=None, dv=None):
+                           impl: str = "auto", dq=None, dk=None, dv=None, deterministic=False):
     """Backward of the varlen zig-zag schedule: each document's chunk pairs
     through zigzag_backward against the document's merged out / lse rows.
     Returns (dq, dk, dv) in q's dtype."""
@@ -222,5 +224,6 @@ def varlen_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cu_se
         zigzag_backward(grad_out[:, a:b], q[:, a:b], cache_k[:, :, a:b], cache_v[:, :, a:b],
                         out[:, a:b], lse[:, :, a:b], scale, cp, impl=impl, dq=dq[:, a:b],
                         dk=dk[:, :, a:b], dv=dv[:, :, a:b],
-                        acc32=(dq32[:, a:b], dk32[:, :, a:b], dv32[:, :, a:b]))
+                        acc32=(dq32[:, a:b], dk32[:, :, a:b], dv32[:, :, a:b]),
+                        deterministic=deterministic)
     return dq, dk, dv

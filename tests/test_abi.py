@@ -159,13 +159,3 @@ def test_empty_query_range_needs_no_buffers_on_host():
     p.cache_k = p.cache_v = None  # no keys: allowed, the rows get lse = -inf
     p.q = None                    # but rows need their buffers
     assert _lib.STATUS[_lib.load().eagle_attn_fwd(ctypes.byref(p), None)] == "EAGLE_ATTN_ERR_NULL"
-
-
-def test_mma_rate_probe_builds_and_exports():
-    """The tcgen05 issue-rate probe compiles for sm_100a and exports its entry point."""
-    import ctypes
-
-    from online_softmax_merge_eagle_b200.probe import mma_rate
-
-    lib = ctypes.CDLL(mma_rate.build())
-    assert hasattr(lib, "mma_rate_probe")

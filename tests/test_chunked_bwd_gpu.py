@@ -85,3 +85,17 @@ def test_chunked_bwd_fullsize_equals_unchunked():
     assert ea.get_status() == 0
     for a, b in ((dq, rq), (dk, rk), (dv, rv)):
         assert (a.float() - b.float()).abs().max().item() <= TB["grad"]
+    # the oracle on the causal prefix of two chunks (rows 0 .. 16383, across the
+    # first chunk edge), two heads: a row's dq and its diagonal blocks' dk / dv
+    # depend only on keys at or before it, so the prefix problem gives them
+    # exactly (block-0 dk / dv of a key need every later row: checked above
+    # against the unchunked path, which the full-size slice tests pin)
+    n = 2 * (131072 // 16)
+    sl = lambda x: x.detach().double().cpu().numpy()  # noqa: E731
+    for h in (0, 7):
+        oq, ok_, ov = oracle.bwd(sl(q[:, :n, h:h + 1]), sl(k[:, :, :n, h:h + 1]),
+                                 sl(v[:, :, :n, h:h + 1]), sl(g[:, :n, h:h + 1]), scale)
+        assert max_abs(dq[:, :n, h:h + 1], oq) <= TB["grad"], h
+        assert max_abs(rq[:, :n, h:h + 1], oq) <= TB["grad"], h  # the unchunked path too
+        assert max_abs(dk[:, 1:, :n, h:h + 1], ok_[:, 1:]) <= TB["grad"], h
+        assert max_abs(dv[:, 1:, :n, h:h + 1], ov[:, 1:]) <= TB["grad"], h

@@ -81,3 +81,22 @@ def test_varlen_zigzag_fullsize_equals_packed():
     assert (lse - rl).abs().max().item() <= TB["lse"]
     for a, b in ((dq, rq), (dk, rk), (dv, rv)):
         assert (a.float() - b.float()).abs().max().item() <= TB["grad"]
+    # documents never see each other, so a whole document is a problem of its
+    # own: the oracle checks every row and key of the two shortest documents
+    # and of the first one (chunk edges included), for two heads
+    lens = np.diff(np.asarray(cu_h))
+    pick = sorted(set(np.argsort(lens)[:2].tolist() + [0]))
+    for d in pick:
+        a, b = int(cu_h[d]), int(cu_h[d + 1])
+        for h in (0, w.H - 1):
+            qh = _np(cpu["q"][:, a:b, h:h + 1])
+            kh = _np(cpu["cache_k"][:, :, a:b, h:h + 1])
+            vh = _np(cpu["cache_v"][:, :, a:b, h:h + 1])
+            gh = _np(cpu["grad_out"][:, a:b, h:h + 1])
+            oo, ol = oracle.fwd(qh, kh, vh, w.scale)
+            oq, ok_, ov = oracle.bwd(qh, kh, vh, gh, w.scale)
+            assert max_abs(out[:, a:b, h:h + 1], oo) <= TB["out"], (d, h)
+            assert max_abs(lse[:, h:h + 1, a:b], ol) <= TB["lse"], (d, h)
+            assert max_abs(dq[:, a:b, h:h + 1], oq) <= TB["grad"], (d, h)
+            assert max_abs(dk[:, :, a:b, h:h + 1], ok_) <= TB["grad"], (d, h)
+            assert max_abs(dv[:, :, a:b, h:h + 1], ov) <= TB["grad"], (d, h)
