@@ -409,7 +409,7 @@ def time_steps(step, steps, warmup, world, ea):
             a, b = pr[key]
             try:
                 vals.append(a.elapsed_time(b))
-            except RuntimeError:  # never recorded (e.g. no backward)
+            except (RuntimeError, ValueError):  # never recorded (e.g. no backward)
                 return 0.0
         return statistics.mean(vals)
     kern = {"fwd_ms": mean_ms("fwd"), "bwd_block0_ms": mean_ms("bwd"),
