@@ -340,13 +340,15 @@ def make_step(args, w, ea, inp, inp_cpu, dev):
             cu_h = inp_cpu["cu_seqlens"]
             rec(prof, "fwd", 0)
             varlen_zigzag_forward(q, k, v, w.scale, cu_h, cp=w.chunks // 2,
-                                  impl=args.kernel_impl, out=out, lse=lse)
+                                  impl=args.kernel_impl, out=out, lse=lse,
+                                  single_launch=w.single_launch)
             rec(prof, "fwd", 1)
             if w.backward:
                 rec(prof, "bwd", 0)
                 varlen_zigzag_backward(g, q, k, v, out, lse, w.scale, cu_h, cp=w.chunks // 2,
                                        impl=args.kernel_impl, dq=dq, dk=dk, dv=dv,
-                                       deterministic=det)
+                                       deterministic=det,
+                                       single_launch=w.single_launch and not det)
                 rec(prof, "bwd", 1)
             return
         if w.chunks:
@@ -358,7 +360,8 @@ def make_step(args, w, ea, inp, inp_cpu, dev):
             if w.backward:
                 rec(prof, "bwd", 0)
                 zigzag_backward(g, q, k, v, out, lse, w.scale, cp=w.chunks // 2,
-                                impl=args.kernel_impl, dq=dq, dk=dk, dv=dv, deterministic=det)
+                                impl=args.kernel_impl, dq=dq, dk=dk, dv=dv, deterministic=det,
+                                single_launch=w.single_launch and not det)
                 rec(prof, "bwd", 1)
             return
         ea.fwd(q, k, v, w.scale, out=out, lse=lse, prof=None if prof is None else prof["fwd"],
@@ -611,11 +614,13 @@ def e2e_measure(args, w, inp, kw, ea, dev, fl, world):
             from online_softmax_merge_eagle_b200.schedules import (varlen_zigzag_backward,
                                                                    varlen_zigzag_forward)
             varlen_zigzag_forward(d["q"], d["cache_k"], d["cache_v"], w.scale, inp["cu_seqlens"],
-                                  cp=w.chunks // 2, out=o["out"], lse=o["lse"])
+                                  cp=w.chunks // 2, out=o["out"], lse=o["lse"],
+                                  single_launch=w.single_launch)
             if w.backward:
                 varlen_zigzag_backward(d["grad_out"], d["q"], d["cache_k"], d["cache_v"],
                                        o["out"], o["lse"], w.scale, inp["cu_seqlens"],
-                                       cp=w.chunks // 2, dq=o["dq"], dk=o["dk"], dv=o["dv"])
+                                       cp=w.chunks // 2, dq=o["dq"], dk=o["dk"], dv=o["dv"],
+                                       single_launch=w.single_launch)
         elif w.chunks:
             from online_softmax_merge_eagle_b200.schedules import zigzag_backward, zigzag_forward
             zigzag_forward(d["q"], d["cache_k"], d["cache_v"], w.scale, cp=w.chunks // 2,
@@ -623,7 +628,7 @@ def e2e_measure(args, w, inp, kw, ea, dev, fl, world):
             if w.backward:
                 zigzag_backward(d["grad_out"], d["q"], d["cache_k"], d["cache_v"], o["out"],
                                 o["lse"], w.scale, cp=w.chunks // 2, dq=o["dq"], dk=o["dk"],
-                                dv=o["dv"])
+                                dv=o["dv"], single_launch=w.single_launch)
         else:
             ea.fwd(d["q"], d["cache_k"], d["cache_v"], w.scale, out=o["out"], lse=o["lse"], **kw)
             if w.backward:

@@ -56,7 +56,7 @@ extern "C" {
  * name, never by position (cf. page "eagle.ring_attention",
  * require_flash_attn_version: positional binding across releases silently
  * binds arguments to the wrong slots). */
-#define EAGLE_ATTN_ABI_VERSION 3
+#define EAGLE_ATTN_ABI_VERSION 4
 
 typedef enum eagle_attn_status {
     EAGLE_ATTN_OK = 0,
@@ -81,7 +81,7 @@ typedef enum eagle_attn_status {
 #define EAGLE_ATTN_DEV_DOC_TOO_LONG 2     /* a document is longer than max_seqlen */
 #define EAGLE_ATTN_DEV_POS_OUTSIDE 3      /* a query or key position lies past cu_seqlens[num_docs] */
 #define EAGLE_ATTN_DEV_TIMEOUT 4          /* a pipeline wait gave up (a library bug; no input causes it) */
-#define EAGLE_ATTN_DEV_BAD_TILE 5         /* a q_tiles entry is negative, >= Tq or not a multiple of 128 */
+#define EAGLE_ATTN_DEV_BAD_TILE 5         /* a q_tiles / q_tile_rows entry out of range, misaligned or out of order */
 #define EAGLE_ATTN_DEV_SMEM_ALIGN 6       /* dynamic shared memory not 1024-byte aligned (a library bug) */
 
 typedef enum eagle_attn_dtype {
@@ -153,15 +153,32 @@ typedef struct eagle_attn_params {
 
     int32_t grad_mode;         /* eagle_attn_grad_mode (backward) */
 
-    /* Forward, tensor-core path: optional device int32 list of num_q_tiles query
-     * row starts (each a multiple of 128 in [0, Tq)).  When set, the forward
-     * computes exactly those 128-row tiles (rows past Tq ignored), one CTA
-     * each in list order, and leaves every other row of out and lse untouched:
-     * one launch serves an emulated rank's rows of a chunk schedule, its key
-     * chunks merged inside the kernel.  A bad entry raises
+    /* Tensor-core path: optional device int32 list of num_q_tiles query row
+     * starts.  Without q_tile_rows each is a multiple of 128 in [0, Tq) and names
+     * a 128-row tile (rows past Tq ignored).  The forward computes exactly those
+     * tiles, one CTA each in list order, and leaves every other row of out and
+     * lse untouched: one launch serves an emulated rank's rows of a chunk
+     * schedule, its key chunks merged inside the kernel.  A bad entry raises
      * EAGLE_ATTN_DEV_BAD_TILE and that tile is skipped.  NULL = all rows. */
     const int32_t *q_tiles;
     int32_t num_q_tiles;
+
+    /* ABI 4.  Optional device int32 list of num_q_tiles row counts, 1 .. 128, one
+     * per q_tiles entry: entry i then names rows [q_tiles[i], q_tiles[i] +
+     * q_tile_rows[i]) with no alignment (start + rows <= Tq), so segments of
+     * documents of any length can be listed (page "eagle.zigzag_ring_attention",
+     * get_half_index: a rank's front and back half of every document).
+     *   Forward: computes exactly those rows, one CTA per entry.
+     *   Backward (tensor-core path, deterministic = 0; q_tiles with or without
+     *   q_tile_rows): entries sorted by start and disjoint; the gradients of the
+     *   loss through exactly those rows' outputs -- dq of those rows (the other
+     *   rows of dq untouched) and their contributions to dk, dv (block 0, and the
+     *   diagonal blocks of those rows; the other rows of the diagonal blocks
+     *   untouched).  With EAGLE_ATTN_GRAD_ACCUMULATE_F32, one call per emulated
+     *   rank sums a chunk schedule's backward.  A list out of range or out of
+     *   order raises EAGLE_ATTN_DEV_BAD_TILE (entries out of range are skipped).
+     * NULL = whole 128-row tiles as above. */
+    const int32_t *q_tile_rows;
 } eagle_attn_params;
 
 /* Returns EAGLE_ATTN_ABI_VERSION of the loaded library. */

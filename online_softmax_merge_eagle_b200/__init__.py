@@ -25,7 +25,7 @@ from ._lib import BF16, F32, GRAD_ACCUMULATE_F32, IMPL, Params
 __all__ = [
     "EagleAttnError", "fwd", "bwd", "merge_out_lse", "merge_diag", "finalize", "get_status",
     "clear_status", "bwd_workspace_size", "eagle_attention", "library_path", "launch_count",
-    "bwd_noalloc",
+    "bwd_noalloc", "query_segments",
 ]
 
 library_path = _lib.LIB_PATH
@@ -127,14 +127,44 @@ def _prof(p, prof):
         p.prof_start, p.prof_stop = prof[0].cuda_event, prof[1].cuda_event
 
 
+def _set_tiles(p, q_tiles, q_tile_rows):
+    """q_tiles / q_tile_rows (int32 CUDA tensors of the same length) into *p."""
+    if q_tiles is None:
+        if q_tile_rows is not None:
+            raise ValueError("q_tile_rows needs q_tiles")
+        return
+    for t in (q_tiles, q_tile_rows):
+        if t is not None and (t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("q_tiles / q_tile_rows must be contiguous int32 CUDA tensors")
+    if q_tile_rows is not None and q_tile_rows.numel() != q_tiles.numel():
+        raise ValueError("q_tile_rows needs one entry per q_tiles entry")
+    p.q_tiles, p.num_q_tiles = q_tiles.data_ptr(), q_tiles.numel()
+    if q_tile_rows is not None:
+        p.q_tile_rows = q_tile_rows.data_ptr()
+
+
+def query_segments(row_ranges, device) -> tuple[torch.Tensor, torch.Tensor]:
+    """(q_tiles, q_tile_rows) for the union of half-open row ranges [a, b):
+    sorted, disjoint segments of at most 128 rows (ranges must not overlap)."""
+    starts, rows = [], []
+    for a, b in sorted(row_ranges):
+        for t in range(a, b, 128):
+            starts.append(t)
+            rows.append(min(128, b - t))
+    return (torch.tensor(starts, dtype=torch.int32).to(device, non_blocking=True),
+            torch.tensor(rows, dtype=torch.int32).to(device, non_blocking=True))
+
+
 def fwd(q, cache_k, cache_v, scale=None, cu_seqlens=None, max_seqlen=None, q_pos_offset=0,
         k_pos_offset=0, causal=True, out_dtype=None, impl="auto", out=None, lse=None, prof=None,
-        q_tiles=None):
+        q_tiles=None, q_tile_rows=None):
     """Forward: returns (out [B,Tq,H,D], lse [B,H,Tq] fp32).  ``out_dtype``
     torch.float32 keeps the block unrounded for a later merge.  ``prof`` =
     (start, stop) torch.cuda.Event pair recorded around the main kernel.
     ``q_tiles``: int32 CUDA tensor of query row starts (multiples of 128); only
-    those 128-row tiles are computed, the other rows of out / lse untouched."""
+    those 128-row tiles are computed, the other rows of out / lse untouched.
+    With ``q_tile_rows`` (rows per entry, 1..128) the starts need no alignment:
+    segments of any length (``query_segments`` builds them from row ranges)."""
     p, cu = _params(q, cache_k, cache_v, scale, cu_seqlens, max_seqlen, q_pos_offset,
                     k_pos_offset, causal, impl)
     od = q.dtype if out_dtype is None else out_dtype
@@ -148,10 +178,7 @@ def fwd(q, cache_k, cache_v, scale=None, cu_seqlens=None, max_seqlen=None, q_pos
     if not lse.is_contiguous() or lse.shape != (p.B, p.H, p.Tq):
         raise ValueError("lse must be a contiguous fp32 [B, H, Tq] tensor")
     p.out, p.lse = out.data_ptr(), lse.data_ptr()
-    if q_tiles is not None:
-        if q_tiles.dtype != torch.int32 or not q_tiles.is_cuda or not q_tiles.is_contiguous():
-            raise ValueError("q_tiles must be a contiguous int32 CUDA tensor")
-        p.q_tiles, p.num_q_tiles = q_tiles.data_ptr(), q_tiles.numel()
+    _set_tiles(p, q_tiles, q_tile_rows)
     _prof(p, prof)
     _check(_lib.load().eagle_attn_fwd(ctypes.byref(p), _stream()), "eagle_attn_fwd")
     return out, lse
@@ -166,11 +193,14 @@ def bwd_workspace_size(q, cache_k, cache_v, **kw) -> int:
 
 def bwd(grad_out, q, cache_k, cache_v, out, lse, scale=None, cu_seqlens=None, max_seqlen=None,
         q_pos_offset=0, k_pos_offset=0, causal=True, deterministic=False, impl="auto",
-        workspace=None, dq=None, dk=None, dv=None, prof=None, grad_accumulate=False):
+        workspace=None, dq=None, dk=None, dv=None, prof=None, grad_accumulate=False,
+        q_tiles=None, q_tile_rows=None):
     """Backward against the MERGED (out, lse): returns (dq, dk, dv) with dk/dv
     covering every block.  ``grad_accumulate``: dq/dk/dv are given fp32 buffers
     (q's / cache_k's element strides) and the call adds its gradient to them
-    (EAGLE_ATTN_GRAD_ACCUMULATE_F32, the chunked schedule's mode)."""
+    (EAGLE_ATTN_GRAD_ACCUMULATE_F32, the chunked schedule's mode).
+    ``q_tiles`` / ``q_tile_rows``: sorted, disjoint query segments; only those
+    rows' part of the gradient (their dq, their contributions to dk / dv)."""
     p, cu = _params(q, cache_k, cache_v, scale, cu_seqlens, max_seqlen, q_pos_offset,
                     k_pos_offset, causal, impl)
     if not _same_layout(grad_out, q) or not _same_layout(out, q):
@@ -195,6 +225,7 @@ def bwd(grad_out, q, cache_k, cache_v, out, lse, scale=None, cu_seqlens=None, ma
         dv = torch.empty_strided(cache_k.shape, cache_k.stride(), dtype=q.dtype, device=q.device)
     p.out, p.lse, p.grad_out = out.data_ptr(), lse.data_ptr(), grad_out.data_ptr()
     p.dq, p.dk, p.dv = dq.data_ptr(), dk.data_ptr(), dv.data_ptr()
+    _set_tiles(p, q_tiles, q_tile_rows)
     lib = _lib.load()
     need = int(lib.eagle_attn_bwd_workspace_size(ctypes.byref(p)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:

@@ -11,7 +11,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libeagleattn.so")
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 
 OK = 0
 STATUS = {
@@ -69,6 +69,7 @@ class Params(ctypes.Structure):
         ("prof_start", ctypes.c_void_p), ("prof_stop", ctypes.c_void_p),
         ("grad_mode", ctypes.c_int32),
         ("q_tiles", ctypes.c_void_p), ("num_q_tiles", ctypes.c_int32),
+        ("q_tile_rows", ctypes.c_void_p),
     ]
 
 

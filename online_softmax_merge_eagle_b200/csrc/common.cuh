@@ -140,6 +140,22 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Query segment i of a q_tiles list: rows [t0, t0 + n).  False (and the CTA or
+// warp skips it) when the entry is out of range: t0 outside [0, Tq), n outside
+// 1 .. 128, t0 + n past Tq, or, for a list without row counts, t0 not a
+// multiple of 128.
+__device__ __forceinline__ bool q_segment(const int32_t *starts, const int32_t *rows, int i,
+                                          int Tq, int &t0, int &n) {
+    t0 = __ldg(starts + i);
+    if (t0 < 0 || t0 >= Tq) return false;
+    if (rows) {
+        n = __ldg(rows + i);
+        return n >= 1 && n <= 128 && n <= Tq - t0;
+    }
+    n = Tq - t0 < 128 ? Tq - t0 : 128;
+    return (t0 & 127) == 0;
+}
+
 // Kernel-side view of the problem (strides in elements).
 struct Problem {
     int B, Tq, Tk, H, D, NB;
@@ -147,7 +163,9 @@ struct Problem {
     int64_t q_sb, q_st;             // q, out, grad_out, dq
     int64_t kv_sb, kv_sblk, kv_st;  // cache_k, cache_v, dk, dv
     int grad_accum;                 // backward: dq/dk/dv are fp32 and the call adds into them
-    const int32_t *q_tiles;         // forward: the query tiles to compute, or null (all)
+    const int32_t *q_tiles;         // the query tiles / segments to compute, or null (all)
+    const int32_t *q_tile_rows;     // rows of each q_tiles entry, or null (128-row tiles)
+    int num_q_tiles;
     MaskDesc mask;
 };
 

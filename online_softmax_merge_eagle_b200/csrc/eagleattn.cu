@@ -80,8 +80,11 @@ int resolve(const eagle_attn_params *p, bool bwd, Resolved *r) {
     P.B = p->B; P.Tq = p->Tq; P.Tk = p->Tk; P.H = p->H; P.D = p->D; P.NB = p->num_blocks;
     P.scale = p->scale;
     P.grad_accum = (bwd && p->grad_mode == EAGLE_ATTN_GRAD_ACCUMULATE_F32) ? 1 : 0;
-    P.q_tiles = bwd ? nullptr : p->q_tiles;
-    if (!bwd && p->q_tiles && p->num_q_tiles < 0) return EAGLE_ATTN_ERR_SHAPE;
+    P.q_tiles = p->q_tiles;
+    P.q_tile_rows = p->q_tiles ? p->q_tile_rows : nullptr;
+    P.num_q_tiles = p->q_tiles ? p->num_q_tiles : 0;
+    if (p->q_tiles && p->num_q_tiles < 0) return EAGLE_ATTN_ERR_SHAPE;
+    if (p->q_tile_rows && !p->q_tiles) return EAGLE_ATTN_ERR_SHAPE;
     const int64_t HD = (int64_t)p->H * p->D;
     P.q_st = p->q_stride_t ? p->q_stride_t : HD;
     P.q_sb = p->q_stride_b ? p->q_stride_b : (int64_t)p->Tq * P.q_st;
@@ -118,8 +121,9 @@ int resolve(const eagle_attn_params *p, bool bwd, Resolved *r) {
     r->tc = (p->impl == EAGLE_ATTN_IMPL_TENSOR_CORE) || (p->impl == EAGLE_ATTN_IMPL_AUTO && tc_ok);
     // fp32 accumulation of the gradients is served by the tensor-core backward only
     if (P.grad_accum && !r->tc) return EAGLE_ATTN_ERR_UNSUPPORTED;
-    // so is a query-tile list
+    // so is a query-tile list; in the backward, by the five-product kernel only
     if (P.q_tiles && !r->tc) return EAGLE_ATTN_ERR_UNSUPPORTED;
+    if (bwd && P.q_tiles && p->deterministic) return EAGLE_ATTN_ERR_UNSUPPORTED;
     return EAGLE_ATTN_OK;
 }
 
@@ -224,7 +228,7 @@ template <int D>
 int dq_finalize_launch(const Problem &P, const eagle_attn_params *p, const float *dq_acc,
                        cudaStream_t s) {
     constexpr int E = D / 32;
-    const int64_t rows = rows_of(P);
+    const int64_t rows = row_slots(P);
     if (rows == 0) return EAGLE_ATTN_OK;
     dim3 grid((unsigned)((rows + 7) / 8));
     if (P.grad_accum)
@@ -258,7 +262,7 @@ int tc_bwd_run(const Problem &P, const eagle_attn_params *p, const float *Dws, f
         if (!make_tmap_f32_2d(&tdq, dq_acc, (uint64_t)D, (uint64_t)acc_rows, kvq::DQ_BOX_COLS,
                               kvq::DQ_BOX_ROWS))
             return EAGLE_ATTN_ERR_CUDA;
-        auto k = kvq::dkdvdq_kernel<D>;
+        auto k = P.q_tiles ? kvq::dkdvdq_kernel<D, true> : kvq::dkdvdq_kernel<D, false>;
         const int sm = kvq::Cfg<D>::SMEM;
         if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, sm) !=
             cudaSuccess)
@@ -358,8 +362,12 @@ int bwd_all(const Problem &P, const eagle_attn_params *p, bool tc, cudaStream_t 
         // tensor-core path: one row pass (D_t, diagonal grads, sum_i dz_i k_i
         // into the dQ workspace, zeros there without diagonal blocks when the
         // five-product kernel adds into it), then the block-0 kernels
-        const int64_t rows = rows_of(P);
+        const int64_t rows = row_slots(P);
         const int zero_dq = p->deterministic ? 0 : 1;
+        if (P.q_tiles && P.num_q_tiles > 0) {  // the list's order, on the device
+            check_segments_kernel<<<1, 256, 0, s>>>(P);
+            if (after_launch()) return EAGLE_ATTN_ERR_CUDA;
+        }
         if (rows > 0) {
             dim3 grid((unsigned)((rows + 7) / 8));
             if (P.grad_accum)
@@ -485,6 +493,8 @@ int attn_merge_diag(const eagle_attn_params *p, void *stream) {
     if (tmp.out_dtype != EAGLE_ATTN_F32) return EAGLE_ATTN_ERR_DTYPE;
     tmp.impl = EAGLE_ATTN_IMPL_GENERIC;
     tmp.cu_seqlens = nullptr;
+    tmp.q_tiles = nullptr;  // every row of the running state
+    tmp.q_tile_rows = nullptr;
     Resolved r;
     int rc = resolve(&tmp, false, &r);
     if (rc) return rc;

@@ -179,6 +179,47 @@ template <> struct RowIO<float, 4> {
 
 constexpr int ROW_THREADS = 256;  // 8 warps, one row each
 
+// Row (b, t, h) of flat warp index idx over all rows ([B, Tq, H], h fastest) or,
+// with a q_tiles list, over B x segments x 128 x H (rows past a segment's count,
+// and segments out of range, give false).
+__device__ __forceinline__ bool row_of(const Problem &P, int64_t idx, int &b, int &t, int &h) {
+    h = (int)(idx % P.H);
+    if (!P.q_tiles) {
+        if (idx >= (int64_t)P.B * P.Tq * P.H) return false;
+        t = (int)((idx / P.H) % P.Tq);
+        b = (int)(idx / ((int64_t)P.H * P.Tq));
+        return true;
+    }
+    const int r = (int)((idx / P.H) % 128);
+    const int64_t bs = idx / ((int64_t)P.H * 128);
+    if (bs >= (int64_t)P.B * P.num_q_tiles) return false;
+    const int seg = (int)(bs % P.num_q_tiles);
+    b = (int)(bs / P.num_q_tiles);
+    int t0, n;
+    if (!q_segment(P.q_tiles, P.q_tile_rows, seg, P.Tq, t0, n) || r >= n) return false;
+    t = t0 + r;
+    return true;
+}
+
+// Warps (rows) a row kernel covers: every row, or 128 per listed segment.
+__host__ __device__ inline int64_t row_slots(const Problem &P) {
+    return P.q_tiles ? (int64_t)P.B * P.num_q_tiles * 128 * P.H : (int64_t)P.B * P.Tq * P.H;
+}
+
+// Checks a q_tiles list for the backward: every entry in range (q_segment) and
+// the segments sorted by start and disjoint.  Raises EAGLE_ATTN_DEV_BAD_TILE.
+__global__ void check_segments_kernel(Problem P) {
+    for (int i = threadIdx.x; i < P.num_q_tiles; i += blockDim.x) {
+        int t0, n, t1, n1;
+        if (!q_segment(P.q_tiles, P.q_tile_rows, i, P.Tq, t0, n)) {
+            raise_status(EAGLE_ATTN_DEV_BAD_TILE);
+        } else if (i + 1 < P.num_q_tiles && q_segment(P.q_tiles, P.q_tile_rows, i + 1, P.Tq, t1, n1) &&
+                   t1 < t0 + n) {
+            raise_status(EAGLE_ATTN_DEV_BAD_TILE);
+        }
+    }
+}
+
 // Fold diagonal blocks 1..NB-1 into the fp32 running state (NeMo AutoModel
 // "eagle.ring_attention", _merge_diag: a one-key block has lse = its logit
 // (Q_t . K_i_t) * scale and out = V_i_t).
@@ -335,19 +376,18 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_diag_kernel(
 // _CachedRingAttention: "the diagonal grads are added in closed form".)
 // dk / dv of the diagonal blocks in GT: T (written), or fp32 with P.grad_accum
 // (added to what the buffers hold).  With zero_dq, dq_diag is written (zeros)
-// also when there are no diagonal blocks.
+// also when there are no diagonal blocks.  With a q_tiles list, the listed rows
+// only.
 template <typename T, typename TO, typename GT, int E>
 __global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
     Problem P, const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ dout, const TO *__restrict__ out, const float *__restrict__ lse,
     float *__restrict__ Dws, float *__restrict__ dq_diag, GT *__restrict__ dk,
     GT *__restrict__ dv, int zero_dq) {
-    int64_t row = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
+    const int64_t idx = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= (int64_t)P.B * P.Tq * P.H) return;
-    const int h = (int)(row % P.H);
-    const int t = (int)((row / P.H) % P.Tq);
-    const int b = (int)(row / ((int64_t)P.H * P.Tq));
+    int b, t, h;
+    if (!row_of(P, idx, b, t, h)) return;
     const int64_t qo = b * P.q_sb + t * P.q_st + (int64_t)h * P.D + lane * E;
     const int64_t li = ((int64_t)b * P.H + h) * P.Tq + t;
     float qf[E], g[E], o[E], acc[E];
@@ -410,17 +450,15 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
 // dq_t = scale * dq_acc_t, the fp32 accumulator ([B, H, Tq, D]) that the
 // five-product backward added its dS K products to (it started from the
 // diagonal blocks' sum_i dz_i k_i): written in GT, or added to the fp32 dq
-// with P.grad_accum.
+// with P.grad_accum.  With a q_tiles list, the listed rows only.
 template <typename GT, int E>
 __global__ void __launch_bounds__(ROW_THREADS) dq_finalize_kernel(Problem P,
                                                                  const float *__restrict__ dq_acc,
                                                                  GT *__restrict__ dq) {
-    int64_t row = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
+    const int64_t idx = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= (int64_t)P.B * P.Tq * P.H) return;
-    const int h = (int)(row % P.H);
-    const int t = (int)((row / P.H) % P.Tq);
-    const int b = (int)(row / ((int64_t)P.H * P.Tq));
+    int b, t, h;
+    if (!row_of(P, idx, b, t, h)) return;
     const int64_t qo = b * P.q_sb + t * P.q_st + (int64_t)h * P.D + lane * E;
     const int64_t li = ((int64_t)b * P.H + h) * P.Tq + t;
     float a[E];

@@ -792,7 +792,9 @@ __device__ __forceinline__ void ew_sync() {
     asm volatile("bar.sync 2, %0;" ::"n"(EW_THREADS) : "memory");
 }
 
-template <int D>
+// SEG: the query slices are the segments of a q_tiles list (a separate
+// instantiation, so that the whole-row path keeps its register allocation).
+template <int D, bool SEG>
 __global__ void __launch_bounds__(THREADS, 1)
     dkdvdq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -829,7 +831,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ks = blockIdx.x * BN, h = blockIdx.y, b = blockIdx.z;
     int tbeg, tend;
     keys_row_range(P.mask, ks, min(ks + BN, P.Tk) - 1, tbeg, tend);
-    const int nsteps = tend >= tbeg ? (tend - tbeg + BM) / BM : 0;
+    // query slices: 128 rows at a time from tbeg or, with a q_tiles list, the
+    // listed segments (sorted, disjoint, <= 128 rows) that meet [tbeg, tend]
+    int seg0 = 0, nsteps = tend >= tbeg ? (tend - tbeg + BM) / BM : 0;
+    if (SEG) {
+        auto seg_start = [&](int i) { return __ldg(P.q_tiles + i); };
+        auto seg_end = [&](int i) {  // one past the last row (search only; entries checked below)
+            return __ldg(P.q_tiles + i) + (P.q_tile_rows ? __ldg(P.q_tile_rows + i) : BM);
+        };
+        int lo = 0, hi = P.num_q_tiles;  // first segment ending after tbeg
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (seg_end(mid) > tbeg) hi = mid; else lo = mid + 1;
+        }
+        seg0 = lo;
+        hi = P.num_q_tiles;  // first segment starting after tend
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (seg_start(mid) > tend) hi = mid; else lo = mid + 1;
+        }
+        nsteps = tend >= tbeg ? lo - seg0 : 0;
+    }
+    // rows [t0, t1] of slice i (t1 - t0 < 128; empty for an entry out of range,
+    // whose rows are then all invisible)
+    auto slice = [&](int i, int &t0, int &t1) {
+        if (!SEG) {
+            t0 = tbeg + i * BM;
+            t1 = min(t0 + BM - 1, tend);
+            return;
+        }
+        int a, n;
+        if (!q_segment(P.q_tiles, P.q_tile_rows, seg0 + i, P.Tq, a, n)) {
+            t0 = tbeg;
+            t1 = tbeg - 1;
+            return;
+        }
+        t0 = max(a, tbeg);
+        t1 = min(a + n - 1, tend);
+        if (t1 < t0) { t0 = tbeg; t1 = tbeg - 1; }
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NBARS; ++i) mbar_init(&bars[i], 1);
@@ -875,18 +915,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             auto load = [&](bool is_do, int i) {
                 uint64_t *bar = is_do ? bar_of + i % OSL : bar_qf + i % QSL;
                 uint8_t *dst = smem + (is_do ? C::do_off(i) : C::q_off(i));
+                int t0, t1;
+                slice(i, t0, t1);
                 mbar_expect_tx(bar, C::QT);
 #pragma unroll
                 for (int cb = 0; cb < D / 64; ++cb)
-                    tma_load_4d(dst + cb * BM * 128, is_do ? &tm_do : &tm_q, bar, cb * 64, h,
-                                tbeg + i * BM, b);
+                    tma_load_4d(dst + cb * BM * 128, is_do ? &tm_do : &tm_q, bar, cb * 64, h, t0, b);
             };
             int q_issued = 0, o_issued = 0;
             for (; q_issued < QSL && q_issued < nsteps; ++q_issued) load(false, q_issued);
             for (; o_issued < OSL && o_issued < nsteps; ++o_issued) load(true, o_issued);
             for (int i = 0; i < nsteps; ++i) {
                 if (!mbar_wait(bar_stg, i & 1, abort)) break;
-                const int row0 = (b * P.H + h) * P.Tq + tbeg + i * BM;
+                int t0, t1;
+                slice(i, t0, t1);
+                const int row0 = (b * P.H + h) * P.Tq + t0;
 #pragma unroll
                 for (int bx = 0; bx < C::NBOX; ++bx)
                     tma_reduce_add_2d(&tm_dq, smem + C::box_off(i, bx), bx * DQ_BOX_COLS, row0);
@@ -1020,19 +1063,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         };
         auto gather = [&](int i) -> RowData {
             RowData d{-INFINITY, 0.f, 1, 0, 1, 0};
-            const int t0 = tbeg + i * BM;
+            if (tid >= BM || i >= nsteps) return d;
+            int t0, t1;
+            slice(i, t0, t1);
             const int t = t0 + tid;
-            if (tid < BM && i < nsteps && t <= tend && t < P.Tq) {
+            if (t <= t1) {
                 if (row_interval(P.mask, t, d.lo, d.hi) != 0) { d.lo = 1; d.hi = 0; }
                 d.L = __ldg(lse + ((int64_t)b * P.H + h) * P.Tq + t);
                 d.dd = __ldg(Dws + ((int64_t)b * P.H + h) * P.Tq + t);
             }
-            if (tid == 0 && i < nsteps) {
+            if (tid == 0) {
                 // every row of the step valid: the interval ends are monotone, so the
                 // step is fully visible to keys in [lo(last row), hi(first row)]
                 const int tl_ = t0 + BM - 1;
                 int lo1 = 1, hi1 = 0, lo0 = 1, hi0 = 0;
-                if (tl_ <= tend && tl_ < P.Tq && row_interval(P.mask, tl_, lo1, hi1) == 0 &&
+                if (tl_ <= t1 && row_interval(P.mask, tl_, lo1, hi1) == 0 &&
                     row_interval(P.mask, t0, lo0, hi0) == 0) {
                     d.flo = lo1;
                     d.fhi = hi0;

@@ -83,6 +83,21 @@ __device__ __forceinline__ bool group_all(bool v) {
     return r != 0;
 }
 
+// Barrier of the two softmax warps that share TMEM lanes quad * 32 .. + 31 (one per
+// warpgroup; named barrier 2 + quad, 64 threads) that also ANDs `v` over them.
+__device__ __forceinline__ bool pair_all(bool v, int quad) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, 64, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(2 + quad)
+        : "memory");
+    return r != 0;
+}
+
 // Bounded wait used only while draining after an abort (ignores the abort flag).
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = globaltimer();
@@ -139,16 +154,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_qtiles = (P.Tq + BM - 1) / BM;
-    // heaviest causal tiles first, or the caller's tile list (its order)
-    const int t0 = P.q_tiles ? __ldg(P.q_tiles + blockIdx.x) : (n_qtiles - 1 - (int)blockIdx.x) * BM;
-    const int h = blockIdx.y, b = blockIdx.z;
-    if (t0 < 0 || t0 >= P.Tq || t0 % BM) {  // CTA-uniform: nothing allocated yet
-        if (threadIdx.x == 0) raise_status(EAGLE_ATTN_DEV_BAD_TILE);
-        return;
+    // heaviest causal tiles first, or the caller's tile / segment list (its
+    // order): rows [t0, t0 + nrows) of the tile, nrows <= 128
+    int t0 = (n_qtiles - 1 - (int)blockIdx.x) * BM, nrows = min(BM, P.Tq - t0);
+    if (P.q_tiles && !q_segment(P.q_tiles, P.q_tile_rows, blockIdx.x, P.Tq, t0, nrows)) {
+        if (threadIdx.x == 0) raise_status(EAGLE_ATTN_DEV_BAD_TILE);  // CTA-uniform: nothing
+        return;                                                       // allocated yet
     }
+    const int h = blockIdx.y, b = blockIdx.z;
 
     int kbeg, kend;
-    rows_key_range(P.mask, t0, min(t0 + BM, P.Tq) - 1, kbeg, kend);
+    rows_key_range(P.mask, t0, t0 + nrows - 1, kbeg, kend);
     const int ntiles = kend >= kbeg ? (kend - kbeg + BN) / BN : 0;
 
     if (threadIdx.x == 0) {
@@ -283,14 +299,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------ softmax ---
         // thread = (row = TMEM lane, half of the columns); the two halves of a
-        // row agree on the running max through shared memory once per tile
+        // row agree on the running max through shared memory once per tile, the
+        // two warps of those rows meeting at their own named barrier
         const int quad = warp & 3;
         const int eg = (warp - 2) >> 2;
         const int r = quad * 32 + lane;
         const int t = t0 + r;
+        const bool row_ok = r < nrows;  // a row of this tile (the rest: other rows, or past Tq)
         constexpr int HC = BN / EW;  // 64 key columns per thread and tile
         int lo = 1, hi = 0;
-        if (t < P.Tq && row_interval(P.mask, t, lo, hi) != 0) { lo = 1; hi = 0; }
+        if (row_ok && row_interval(P.mask, t, lo, hi) != 0) { lo = 1; hi = 0; }
         const float sl2 = P.scale * 1.4426950408889634f;
         // m: reference max (exp2 domain) of l and O; -inf until the row sees a key
         float m = -INFINITY, l = 0.f;  // l: this half's partial sum
@@ -326,7 +344,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
                 xmax[((j & 1) * EW + eg) * BM + r] = mx;
             }
-            ok = group_all(ok);  // both halves' maxima are in shared memory
+            // both halves of these rows have their maxima in shared memory (the other
+            // rows' warps need not wait for it)
+            ok = pair_all(ok, quad);
             if (!ok) break;
 #pragma unroll
             for (int g = 0; g < EW; ++g) mx = fmaxf(mx, xmax[((j & 1) * EW + g) * BM + r]);
@@ -453,12 +473,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 res[i] = fmaf(__uint_as_float(o[i]), alpha, acc[cc * 32 + i] * beta);
-            if (t < P.Tq && ok) {
+            if (row_ok && ok) {
                 TO *orow = out + b * P.q_sb + (int64_t)t * P.q_st + (int64_t)h * D + c * 32;
                 store_chunk32<TO>(orow, res, inv);
             }
         }
-        if (eg == 0 && t < P.Tq && ok)
+        if (eg == 0 && row_ok && ok)
             lse_out[((int64_t)b * P.H + h) * P.Tq + t] =
                 l_fin > 0.f ? (m_use + __log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
     }

@@ -100,11 +100,24 @@ WORKLOADS: dict[str, Workload] = {
     "chunked_bwd_bf16": Workload("chunked_bwd_bf16", B=1, Tq=131072, H=8, D=128, num_blocks=4,
                                  dtype=torch.bfloat16, chunks=16,
                                  notes="chunked_bf16 forward + the zig-zag chunked backward"),
+    "chunked_bwd_single_bf16": Workload("chunked_bwd_single_bf16", B=1, Tq=131072, H=8, D=128,
+                                        num_blocks=4, dtype=torch.bfloat16, chunks=16,
+                                        single_launch=True,
+                                        notes="chunked_bwd_bf16 with one forward and one "
+                                              "backward launch per emulated rank"),
     "varlen_zigzag_bf16": Workload("varlen_zigzag_bf16", B=1, Tq=32768, H=32, D=128,
                                    num_blocks=4, dtype=torch.bfloat16, chunks=16,
                                    doc_lengths=doc_lengths_multiple(32768, 256, 8192, 16, 0),
                                    notes="varlen_bf16's documents rounded to multiples of 16, "
                                          "each cut into 16 zig-zag chunks (emulated cp=8)"),
+    "varlen_zigzag_single_bf16": Workload("varlen_zigzag_single_bf16", B=1, Tq=32768, H=32,
+                                          D=128, num_blocks=4, dtype=torch.bfloat16, chunks=16,
+                                          doc_lengths=doc_lengths_multiple(32768, 256, 8192, 16,
+                                                                           0),
+                                          single_launch=True,
+                                          notes="varlen_zigzag_bf16 with one forward and one "
+                                                "backward launch per emulated rank over every "
+                                                "document's chunks"),
     "frozen_target_bf16": Workload("frozen_target_bf16", B=1, Tq=8192, H=32, D=128,
                                    num_blocks=1, dtype=torch.bfloat16, Tk=65536,
                                    q_pos_offset=57344, backward=False,

@@ -33,7 +33,7 @@ from __future__ import annotations
 
 import torch
 
-from . import bwd, bwd_workspace_size, finalize, fwd, merge_diag, merge_out_lse
+from . import bwd, bwd_workspace_size, finalize, fwd, merge_diag, merge_out_lse, query_segments
 
 
 def zigzag_owner_chunks(rank: int, cp: int) -> tuple[int, int]:
@@ -113,8 +113,27 @@ def _chunk_schedule_forward(q, cache_k, cache_v, scale, n_chunks, rank_chunks, i
     return out, lse
 
 
+def zigzag_rank_rows(rank: int, cp: int, a: int, b: int) -> list[tuple[int, int]]:
+    """Half-open row ranges of ``rank``'s two chunks of the sequence [a, b) cut into
+    2*cp chunks ("eagle.zigzag_ring_attention", get_half_index: the front and
+    back half that rank r holds)."""
+    c = (b - a) // (2 * cp)
+    return [(a + ch * c, a + (ch + 1) * c) for ch in zigzag_owner_chunks(rank, cp)]
+
+
+def _single_launch_backward(grad_out, q, cache_k, cache_v, out, lse, scale, rank_rows, impl,
+                            dq32, dk32, dv32, **mask):
+    """One backward launch per emulated rank over its query rows (every key
+    they see, in one kernel), summed into fp32 buffers."""
+    for rows in rank_rows:
+        tiles, counts = query_segments(rows, q.device)
+        bwd(grad_out, q, cache_k, cache_v, out, lse, scale, impl=impl, dq=dq32, dk=dk32, dv=dv32,
+            grad_accumulate=True, q_tiles=tiles, q_tile_rows=counts, **mask)
+
+
 def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, impl: str = "auto",
-                    dq=None, dk=None, dv=None, ranks=None, acc32=None, deterministic=False):
+                    dq=None, dk=None, dv=None, ranks=None, acc32=None, deterministic=False,
+                    single_launch: bool = False):
     """Backward of the whole sequence through the zig-zag chunk schedule.
 
     Shapes as zigzag_forward; out / lse are the merged forward results of the
@@ -127,7 +146,9 @@ def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, imp
     dv32): zeroed fp32 accumulators with q's / cache_k's element strides to use
     instead of fresh ones (the varlen schedule passes views of whole-sequence
     buffers).  ``deterministic`` selects the reproducible backward for every
-    pair (eagle_attn_params.deterministic).
+    pair (eagle_attn_params.deterministic).  ``single_launch``: one backward
+    launch per rank over its two query chunks against every key (a segment list
+    in the ABI), instead of one call per chunk pair; not with ``deterministic``.
     """
     B, T, H, D = q.shape
     if B != 1 or T % (2 * cp):
@@ -138,6 +159,14 @@ def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, imp
         acc32 = (torch.zeros(q.shape, **f32), torch.zeros(cache_k.shape, **f32),
                  torch.zeros(cache_k.shape, **f32))
     dq32, dk32, dv32 = acc32
+    if single_launch:
+        if deterministic:
+            raise ValueError("the single-launch backward is the five-product kernel only")
+        _single_launch_backward(grad_out, q, cache_k, cache_v, out, lse, scale,
+                                [zigzag_rank_rows(r, cp, 0, T)
+                                 for r in (range(cp) if ranks is None else ranks)],
+                                impl, dq32, dk32, dv32)
+        return _finalize_grads(q, cache_k, dq32, dk32, dv32, dq, dk, dv)
     lse_c = torch.empty((1, H, c), **f32)
     k0, v0 = cache_k[:, :1], cache_v[:, :1]
     ws = torch.empty(max(1, bwd_workspace_size(q[:, :c], cache_k[:, :, :c], cache_v[:, :, :c],
@@ -159,11 +188,16 @@ def zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cp: int, imp
                     q_pos_offset=qc * c, k_pos_offset=kc * c, impl=impl, workspace=ws,
                     dq=dq32[:, qs], dk=dkk, dv=dvv, grad_accumulate=True,
                     deterministic=deterministic)
+    return _finalize_grads(q, cache_k, dq32, dk32, dv32, dq, dk, dv)
+
+
+def _finalize_grads(q, cache_k, dq32, dk32, dv32, dq, dk, dv):
+    """The fp32 sums cast to q's dtype (into dq / dk / dv when given)."""
     dq = finalize(dq32, q.dtype, out=dq)
     if dk is None:
         dk = torch.empty_like(cache_k)
     if dv is None:
-        dv = torch.empty_like(cache_v)
+        dv = torch.empty_like(cache_k)
     for i in range(cache_k.shape[1]):  # block by block: dk / dv may be views of a larger cache
         finalize(dk32[:, i], q.dtype, out=dk[:, i])
         finalize(dv32[:, i], q.dtype, out=dv[:, i])
@@ -181,13 +215,25 @@ def _doc_bounds(cu_seqlens, T: int, cp: int) -> list[tuple[int, int]]:
     return docs
 
 
+def _packed_mask(cu_seqlens, T, device):
+    """cu_seqlens as a device int32 tensor and the longest document."""
+    cu = [int(x) for x in (cu_seqlens.tolist() if isinstance(cu_seqlens, torch.Tensor)
+                           else list(cu_seqlens))]
+    return (torch.tensor(cu, dtype=torch.int32).to(device, non_blocking=True),
+            max(b - a for a, b in zip(cu, cu[1:])))
+
+
 def varlen_zigzag_forward(q, cache_k, cache_v, scale, cu_seqlens, cp: int, impl: str = "auto",
-                          out=None, lse=None):
+                          out=None, lse=None, single_launch: bool = False, ranks=None):
     """Forward of packed documents through the varlen zig-zag schedule: each
     document's 2*cp chunks through zigzag_forward (the document's positions
     start at 0, so no mask crosses documents).  q [1, T, H, D], cache_k/cache_v
     [1, NB, T, H, D]; cu_seqlens (host sequence or tensor) [num_docs + 1] with
-    every length divisible by 2*cp.  Returns (out, lse) like zigzag_forward."""
+    every length divisible by 2*cp.  Returns (out, lse) like zigzag_forward.
+    ``single_launch``: one launch per emulated rank (or the ``ranks`` listed)
+    over its front and back chunk of every document at once, the packed
+    (cu_seqlens) mask keeping the documents apart -- the pages' one varlen call
+    per ring step over every document's halves."""
     B, T, H, D = q.shape
     if B != 1:
         raise ValueError("the varlen zig-zag schedule is unbatched (B == 1)")
@@ -195,17 +241,29 @@ def varlen_zigzag_forward(q, cache_k, cache_v, scale, cu_seqlens, cp: int, impl:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((1, H, T), dtype=torch.float32, device=q.device)
-    for a, b in _doc_bounds(cu_seqlens, T, cp):
+    docs = _doc_bounds(cu_seqlens, T, cp)
+    if single_launch:
+        cu_d, max_len = _packed_mask(cu_seqlens, T, q.device)
+        for r in (range(cp) if ranks is None else ranks):
+            tiles, counts = query_segments([rr for a, b in docs
+                                            for rr in zigzag_rank_rows(r, cp, a, b)], q.device)
+            fwd(q, cache_k, cache_v, scale, cu_seqlens=cu_d, max_seqlen=max_len, impl=impl,
+                out=out, lse=lse, q_tiles=tiles, q_tile_rows=counts)
+        return out, lse
+    for a, b in docs:
         zigzag_forward(q[:, a:b], cache_k[:, :, a:b], cache_v[:, :, a:b], scale, cp, impl=impl,
                        out=out[:, a:b], lse=lse[:, :, a:b])
     return out, lse
 
 
 def varlen_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cu_seqlens, cp: int,
-                           impl: str = "auto", dq=None, dk=None, dv=None, deterministic=False):
+                           impl: str = "auto", dq=None, dk=None, dv=None, deterministic=False,
+                           single_launch: bool = False):
     """Backward of the varlen zig-zag schedule: each document's chunk pairs
     through zigzag_backward against the document's merged out / lse rows.
-    Returns (dq, dk, dv) in q's dtype."""
+    Returns (dq, dk, dv) in q's dtype.  ``single_launch``: one backward launch
+    per emulated rank over its chunks of every document (packed mask), the
+    ranks' parts summed in fp32; not with ``deterministic``."""
     B, T, H, D = q.shape
     if B != 1:
         raise ValueError("the varlen zig-zag schedule is unbatched (B == 1)")
@@ -220,7 +278,17 @@ def varlen_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, cu_se
     dq32 = torch.zeros(q.shape, **f32)
     dk32 = torch.zeros(cache_k.shape, **f32)
     dv32 = torch.zeros(cache_k.shape, **f32)
-    for a, b in _doc_bounds(cu_seqlens, T, cp):
+    docs = _doc_bounds(cu_seqlens, T, cp)
+    if single_launch:
+        if deterministic:
+            raise ValueError("the single-launch backward is the five-product kernel only")
+        cu_d, max_len = _packed_mask(cu_seqlens, T, q.device)
+        _single_launch_backward(grad_out, q, cache_k, cache_v, out, lse, scale,
+                                [[rr for a, b in docs for rr in zigzag_rank_rows(r, cp, a, b)]
+                                 for r in range(cp)],
+                                impl, dq32, dk32, dv32, cu_seqlens=cu_d, max_seqlen=max_len)
+        return _finalize_grads(q, cache_k, dq32, dk32, dv32, dq, dk, dv)
+    for a, b in docs:
         zigzag_backward(grad_out[:, a:b], q[:, a:b], cache_k[:, :, a:b], cache_v[:, :, a:b],
                         out[:, a:b], lse[:, :, a:b], scale, cp, impl=impl, dq=dq[:, a:b],
                         dk=dk[:, :, a:b], dv=dv[:, :, a:b],

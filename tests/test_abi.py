@@ -77,6 +77,7 @@ def _valid_params():
      "EAGLE_ATTN_ERR_SHAPE"),
     (lambda p: (setattr(p, "q_tiles", 1 << 20), setattr(p, "num_q_tiles", 1),
                 setattr(p, "impl", 2)), "EAGLE_ATTN_ERR_UNSUPPORTED"),   # generic kernels
+    (lambda p: setattr(p, "q_tile_rows", 1 << 20), "EAGLE_ATTN_ERR_SHAPE"),  # rows, no starts
 ])
 def test_fwd_rejects_bad_arguments_on_host(mutate, code):
     p = _valid_params()
@@ -96,6 +97,11 @@ def test_bwd_rejects_missing_workspace():
     lambda p: (setattr(p, "grad_mode", 1), setattr(p, "dtype", _lib.F32),
                setattr(p, "out_dtype", _lib.F32)),                       # fp32 inputs: no TC path
     lambda p: (setattr(p, "grad_mode", 1), setattr(p, "impl", 2)),       # generic kernels
+    # query segments: the five-product kernel only
+    lambda p: (setattr(p, "q_tiles", 1 << 20), setattr(p, "num_q_tiles", 1),
+               setattr(p, "deterministic", 1)),
+    lambda p: (setattr(p, "q_tiles", 1 << 20), setattr(p, "num_q_tiles", 1),
+               setattr(p, "impl", 2)),
 ])
 def test_bwd_rejects_unserved_grad_modes_on_host(mutate):
     p = _valid_params()

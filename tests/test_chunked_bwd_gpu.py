@@ -24,12 +24,17 @@ def _inputs(T, H, D, NB, seed=3):
     return t["q"], t["cache_k"], t["cache_v"], t["grad_out"]
 
 
-@pytest.mark.parametrize("T,H,D,NB,cp", [(1024, 2, 128, 3, 2), (768, 2, 64, 2, 3)])
-def test_chunked_bwd_matches_oracle_and_unchunked(T, H, D, NB, cp):
+@pytest.mark.parametrize("single", [False, True])
+@pytest.mark.parametrize("T,H,D,NB,cp", [(1024, 2, 128, 3, 2), (768, 2, 64, 2, 3),
+                                         (1200, 2, 128, 2, 3)])
+def test_chunked_bwd_matches_oracle_and_unchunked(T, H, D, NB, cp, single):
+    """Per (query chunk, key chunk) pair, or (``single``) one launch per
+    emulated rank over its two chunks (1200 rows, cp 3: chunks of 200 rows,
+    not tile aligned)."""
     q, k, v, g = _inputs(T, H, D, NB)
     scale = D ** -0.5
-    out, lse = zigzag_forward(q, k, v, scale, cp=cp)
-    dq, dk, dv = zigzag_backward(g, q, k, v, out, lse, scale, cp=cp)
+    out, lse = zigzag_forward(q, k, v, scale, cp=cp, single_launch=single and T % 256 == 0)
+    dq, dk, dv = zigzag_backward(g, q, k, v, out, lse, scale, cp=cp, single_launch=single)
     rq, rk, rv = ea.bwd(g, q, k, v, out, lse, scale)
     torch.cuda.synchronize()
     assert ea.get_status() == 0
@@ -73,13 +78,15 @@ def test_grad_accumulate_adds_exactly(deterministic):
 
 
 @pytest.mark.slow
-def test_chunked_bwd_fullsize_equals_unchunked():
+@pytest.mark.parametrize("single", [False, True])
+def test_chunked_bwd_fullsize_equals_unchunked(single):
     """131072 positions, 16 zig-zag chunks (emulated cp = 8), NB = 4, H = 8:
-    every gradient of the chunked backward equals the unchunked one."""
+    every gradient of the chunked backward (per pair, or one launch per rank)
+    equals the unchunked one."""
     q, k, v, g = _inputs(131072, 8, 128, 4, seed=0)
     scale = 128 ** -0.5
-    out, lse = zigzag_forward(q, k, v, scale, cp=8)
-    dq, dk, dv = zigzag_backward(g, q, k, v, out, lse, scale, cp=8)
+    out, lse = zigzag_forward(q, k, v, scale, cp=8, single_launch=single)
+    dq, dk, dv = zigzag_backward(g, q, k, v, out, lse, scale, cp=8, single_launch=single)
     rq, rk, rv = ea.bwd(g, q, k, v, out, lse, scale)
     torch.cuda.synchronize()
     assert ea.get_status() == 0

@@ -55,6 +55,42 @@ def test_varlen_zigzag_matches_packed_and_oracle(docs, H, D, NB, cp):
         assert max_abs(dv[:, :, :, h:h + 1], ov) <= TB["grad"]
 
 
+@pytest.mark.parametrize("docs,H,D,NB,cp", [
+    ([256, 64, 520, 184], 2, 128, 3, 4),
+    ([48, 192, 12, 132], 2, 64, 2, 3),
+])
+def test_varlen_zigzag_single_launch_matches_packed_and_oracle(docs, H, D, NB, cp):
+    """One launch per emulated rank (forward and backward) over its front and
+    back chunk of every document: the packed path and the oracle."""
+    T = sum(docs)
+    t = make_tensors(1, T, H, D, NB, torch.bfloat16, seed=8, device="cuda")
+    q, k, v, g = t["q"], t["cache_k"], t["cache_v"], t["grad_out"]
+    scale = D ** -0.5
+    cu_h = cu_seqlens(docs)
+    cu_d = torch.as_tensor(cu_h, device="cuda")
+    out, lse = varlen_zigzag_forward(q, k, v, scale, cu_h, cp=cp, single_launch=True)
+    dq, dk, dv = varlen_zigzag_backward(g, q, k, v, out, lse, scale, cu_h, cp=cp,
+                                        single_launch=True)
+    ro, rl = ea.fwd(q, k, v, scale, cu_seqlens=cu_d, max_seqlen=max(docs))
+    rq, rk, rv = ea.bwd(g, q, k, v, ro, rl, scale, cu_seqlens=cu_d, max_seqlen=max(docs))
+    torch.cuda.synchronize()
+    assert ea.get_status() == 0
+    assert max_abs(out, _np(ro)) <= TB["out"]
+    assert max_abs(lse, _np(rl)) <= TB["lse"]
+    for a, b in ((dq, rq), (dk, rk), (dv, rv)):
+        assert max_abs(a, _np(b)) <= TB["grad"]
+    for h in (0, H - 1):
+        qh, kh, vh, gh = (_np(q[:, :, h:h + 1]), _np(k[:, :, :, h:h + 1]),
+                          _np(v[:, :, :, h:h + 1]), _np(g[:, :, h:h + 1]))
+        oo, ol = oracle.fwd(qh, kh, vh, scale, cu_seqlens=np.asarray(cu_h))
+        oq, ok_, ov = oracle.bwd(qh, kh, vh, gh, scale, cu_seqlens=np.asarray(cu_h))
+        assert max_abs(out[:, :, h:h + 1], oo) <= TB["out"]
+        assert max_abs(lse[:, h:h + 1], ol) <= TB["lse"]
+        assert max_abs(dq[:, :, h:h + 1], oq) <= TB["grad"]
+        assert max_abs(dk[:, :, :, h:h + 1], ok_) <= TB["grad"]
+        assert max_abs(dv[:, :, :, h:h + 1], ov) <= TB["grad"]
+
+
 def test_varlen_zigzag_rejects_indivisible_documents():
     t = make_tensors(1, 100, 1, 64, 1, torch.bfloat16, grad=False, device="cuda")
     with pytest.raises(ValueError):
@@ -62,7 +98,8 @@ def test_varlen_zigzag_rejects_indivisible_documents():
 
 
 @pytest.mark.slow
-def test_varlen_zigzag_fullsize_equals_packed():
+@pytest.mark.parametrize("single", [False, True])
+def test_varlen_zigzag_fullsize_equals_packed(single):
     """The varlen_zigzag_bf16 workload (T 32768, H 32, NB 4, 11 documents,
     16 chunks each): forward and backward equal the unchunked packed path."""
     w = WORKLOADS["varlen_zigzag_bf16"]
@@ -70,8 +107,10 @@ def test_varlen_zigzag_fullsize_equals_packed():
     q, k, v, g = (cpu[n].cuda() for n in ("q", "cache_k", "cache_v", "grad_out"))
     cu_h = cpu["cu_seqlens"]
     cu_d = torch.as_tensor(cu_h, device="cuda")
-    out, lse = varlen_zigzag_forward(q, k, v, w.scale, cu_h, cp=w.chunks // 2)
-    dq, dk, dv = varlen_zigzag_backward(g, q, k, v, out, lse, w.scale, cu_h, cp=w.chunks // 2)
+    out, lse = varlen_zigzag_forward(q, k, v, w.scale, cu_h, cp=w.chunks // 2,
+                                     single_launch=single)
+    dq, dk, dv = varlen_zigzag_backward(g, q, k, v, out, lse, w.scale, cu_h, cp=w.chunks // 2,
+                                        single_launch=single)
     ro, rl = ea.fwd(q, k, v, w.scale, cu_seqlens=cu_d, max_seqlen=cpu["max_seqlen"])
     rq, rk, rv = ea.bwd(g, q, k, v, ro, rl, w.scale, cu_seqlens=cu_d,
                         max_seqlen=cpu["max_seqlen"])
