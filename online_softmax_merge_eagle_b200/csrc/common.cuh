@@ -35,13 +35,22 @@ struct MaskDesc {
     int Tq, Tk;
 };
 
+// The mask functions below also compile for the host, where a test checks them
+// against a brute-force visibility count.
+#ifdef __CUDA_ARCH__
+#define EAGLE_LDG(p) __ldg(p)
+#else
+#define EAGLE_LDG(p) (*(p))
+#endif
+#define EAGLE_HD __host__ __device__ __forceinline__
+
 // Document holding global position pos (binary search); -1 if none.
-__device__ __forceinline__ int find_doc(const int32_t *cu, int nd, int64_t pos) {
-    if (pos < 0 || pos >= (int64_t)__ldg(cu + nd)) return -1;
+EAGLE_HD int find_doc(const int32_t *cu, int nd, int64_t pos) {
+    if (pos < 0 || pos >= (int64_t)EAGLE_LDG(cu + nd)) return -1;
     int lo = 0, hi = nd - 1;  // invariant: cu[lo] <= pos < cu[hi+1]
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)__ldg(cu + mid) <= pos) lo = mid; else hi = mid - 1;
+        if ((int64_t)EAGLE_LDG(cu + mid) <= pos) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -51,14 +60,14 @@ __device__ __forceinline__ int find_doc(const int32_t *cu, int nd, int64_t pos) 
 // see lies before key 0; +1 = empty because it lies past key Tk-1.  The class
 // is non-decreasing in t (a prefix of -1, then 0, then a suffix of +1) and, on
 // the class-0 rows, lo and hi are non-decreasing in t.
-__device__ __forceinline__ int row_interval(const MaskDesc &m, int t, int &lo, int &hi) {
+EAGLE_HD int row_interval(const MaskDesc &m, int t, int &lo, int &hi) {
     int64_t qp = m.q_off + t;
     int64_t glo = INT64_MIN / 4, ghi = INT64_MAX / 4;
     if (m.cu) {
         int d = find_doc(m.cu, m.num_docs, qp);
         if (d < 0) { lo = 0; hi = -1; return qp < 0 ? -1 : 1; }
-        glo = __ldg(m.cu + d);
-        ghi = (int64_t)__ldg(m.cu + d + 1) - 1;
+        glo = EAGLE_LDG(m.cu + d);
+        ghi = (int64_t)EAGLE_LDG(m.cu + d + 1) - 1;
     }
     if (m.causal && qp < ghi) ghi = qp;
     int64_t l = glo - m.k_off, h = ghi - m.k_off;
@@ -69,53 +78,61 @@ __device__ __forceinline__ int row_interval(const MaskDesc &m, int t, int &lo, i
     return 0;
 }
 
-// Key range [kbeg, kend] touched by query rows [t0, t1]; kend < kbeg if none.
-__device__ __forceinline__ void rows_key_range(const MaskDesc &m, int t0, int t1, int &kbeg,
-                                               int &kend) {
-    int l, h;
-    // ta = first row in [t0, t1] of class >= 0
-    int a = t0, b = t1 + 1;
-    while (a < b) {
-        int mid = (a + b) >> 1;
-        if (row_interval(m, mid, l, h) >= 0) b = mid; else a = mid + 1;
-    }
-    int ta = a;
-    // tb = last row in [t0, t1] of class <= 0
-    a = t0 - 1; b = t1;
-    while (a < b) {
-        int mid = (a + b + 1) >> 1;
-        if (row_interval(m, mid, l, h) <= 0) a = mid; else b = mid - 1;
-    }
-    int tb = a;
-    if (ta > tb || ta > t1 || tb < t0) { kbeg = 0; kend = -1; return; }
-    int c0 = row_interval(m, ta, l, h);
-    kbeg = l;
-    int c1 = row_interval(m, tb, l, h);
-    kend = h;
-    if (c0 != 0 || c1 != 0) { kbeg = 0; kend = -1; }
+// [lo, hi] (global positions) intersected with [0, n): as local indices [a, b]
+// (b < a when empty).
+EAGLE_HD void clip_range(int64_t lo, int64_t hi, int64_t off, int n, int &a, int &b) {
+    lo -= off;
+    hi -= off;
+    if (lo < 0) lo = 0;
+    if (hi > n - 1) hi = n - 1;
+    if (lo > hi) { a = 0; b = -1; return; }
+    a = (int)lo;
+    b = (int)hi;
 }
 
-// Query rows whose interval meets keys [k0, k1]: the contiguous range
-// [tbeg, tend] (tend < tbeg if none).
-__device__ __forceinline__ void keys_row_range(const MaskDesc &m, int k0, int k1, int &tbeg,
-                                               int &tend) {
-    int l, h;
-    // first t with class +1, or class 0 and hi_t >= k0  (a monotone predicate)
-    int a = 0, b = m.Tq;
-    while (a < b) {
-        int mid = (a + b) >> 1;
-        int c = row_interval(m, mid, l, h);
-        if (c > 0 || (c == 0 && h >= k0)) b = mid; else a = mid + 1;
+// Key range [kbeg, kend] seen by query rows [t0, t1] (t0 <= t1); kend < kbeg if
+// none.  A row sees from its document's start (from everything, without
+// documents) to its own position (causal) or its document's end, so the rows of a
+// range see one interval: from the first row's document start to the last row's
+// position or document end.
+EAGLE_HD void rows_key_range(const MaskDesc &m, int t0, int t1, int &kbeg, int &kend) {
+    if (t1 < t0) { kbeg = 0; kend = -1; return; }
+    int64_t a = m.q_off + t0, c = m.q_off + t1;
+    int64_t glo = INT64_MIN / 4, ghi = m.causal ? c : INT64_MAX / 4;
+    if (m.cu) {
+        // rows outside every document see nothing
+        const int64_t end = EAGLE_LDG(m.cu + m.num_docs);
+        if (a < 0) a = 0;
+        if (c > end - 1) c = end - 1;
+        if (a > c) { kbeg = 0; kend = -1; return; }
+        glo = EAGLE_LDG(m.cu + find_doc(m.cu, m.num_docs, a));
+        ghi = m.causal ? c : (int64_t)EAGLE_LDG(m.cu + find_doc(m.cu, m.num_docs, c) + 1) - 1;
     }
-    tbeg = a;
-    // last t with class -1, or class 0 and lo_t <= k1
-    a = -1; b = m.Tq - 1;
-    while (a < b) {
-        int mid = (a + b + 1) >> 1;
-        int c = row_interval(m, mid, l, h);
-        if (c < 0 || (c == 0 && l <= k1)) a = mid; else b = mid - 1;
+    clip_range(glo, ghi, m.k_off, m.Tk, kbeg, kend);
+}
+
+// Query rows [tbeg, tend] that see a key in [k0, k1] (0 <= k0 <= k1 < Tk); tend <
+// tbeg if none.  By the same argument, from the first key's position (causal) or
+// document start to the last key's document end.
+EAGLE_HD void keys_row_range(const MaskDesc &m, int k0, int k1, int &tbeg, int &tend) {
+    if (k1 < k0) { tbeg = 0; tend = -1; return; }
+    int64_t a = m.k_off + k0, c = m.k_off + k1;
+    int64_t glo = m.causal ? a : INT64_MIN / 4, ghi = INT64_MAX / 4;
+    if (m.cu) {
+        const int64_t end = EAGLE_LDG(m.cu + m.num_docs);
+        if (a < 0) a = 0;
+        if (c > end - 1) c = end - 1;
+        if (a > c) { tbeg = 0; tend = -1; return; }
+        glo = m.causal ? a : (int64_t)EAGLE_LDG(m.cu + find_doc(m.cu, m.num_docs, a));
+        ghi = (int64_t)EAGLE_LDG(m.cu + find_doc(m.cu, m.num_docs, c) + 1) - 1;
     }
-    tend = a;
+    clip_range(glo, ghi, m.q_off, m.Tq, tbeg, tend);
+}
+
+// Query rows [ta, tb] that see local key s (empty, tb < ta, for s outside [0, Tk)).
+EAGLE_HD void key_rows(const MaskDesc &m, int s, int &ta, int &tb) {
+    if (s < 0 || s >= m.Tk) { ta = 0; tb = -1; return; }
+    keys_row_range(m, s, s, ta, tb);
 }
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

@@ -107,6 +107,20 @@ __device__ __forceinline__ void tma_reduce_add_2d(const void *tmap, const void *
         "r"(smem_u32(src)), "r"(c0), "r"(c1)
         : "memory");
 }
+// 4-byte asynchronous copy global -> shared (no register holds the value); a
+// thread's copies complete at cp_async_wait_all, and a barrier then makes them
+// visible to the other threads.
+__device__ __forceinline__ void cp_async_4(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

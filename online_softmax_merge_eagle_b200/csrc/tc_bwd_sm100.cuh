@@ -349,9 +349,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                     r_full[1] = next.fhi;
                 }
             }
-            next = gather(i + 1);
             ok = group_all(ok);  // row data written; all element-wise warps agree to go on
             if (!ok) break;
+            next = gather(i + 1);  // after the barrier, which would wait for these loads
             ok = __all_sync(0xffffffffu, mbar_wait(bar_stf, i & 1, abort));
             if (!ok) continue;
             tc_fence_after();
@@ -768,9 +768,9 @@ struct Cfg {
     static constexpr int OFF_Q = OFF_V + KT;
     static constexpr int OFF_DO = OFF_Q + QSL * QT;
     static constexpr int OFF_DS = OFF_DO + OSL * QT;  // own dS^T tile (D = 64 only)
-    static constexpr int OFF_ROW = OFF_DS + (DS_IN_DO ? 0 : DST);  // lse2, D, lo, hi, 2 ints
-    static constexpr int ROW_BYTES = 4 * BM * 4 + 16;
-    static constexpr int OFF_BAR = OFF_ROW + ROW_BYTES;
+    static constexpr int OFF_ROW = OFF_DS + (DS_IN_DO ? 0 : DST);  // two RowSlots
+    static constexpr int ROW_BYTES = 2 * BM * 4 + 16;              // lse, D_t, t0, t1
+    static constexpr int OFF_BAR = OFF_ROW + 2 * ROW_BYTES;
     static constexpr int NBARS = 20;  // >= the barriers laid out in the kernel
     // no realignment slack: the kernel checks that the base is 1024-byte aligned
     static constexpr int SMEM = OFF_BAR + NBARS * 8 + 16;
@@ -819,11 +819,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t *bar_dvd = bar_dpf + 1;       // dV_i done: dO_i no longer read
     uint64_t *bar_dqf = bar_dvd + 1;       // dQ_i in TMEM (dK_i done too: dS^T free)
     uint64_t *bar_ptf = bar_dqf + 1;       // P^T_i written over S^T_i (EW_THREADS)
-    uint64_t *bar_dsf = bar_ptf + 1;       // dS^T_i in shared memory, dP^T_i read (EW_THREADS)
+    uint64_t *bar_dpr = bar_ptf + 1;       // dP^T_i read out of TMEM (EW_THREADS)
+    uint64_t *bar_dsf = bar_dpr + 1;       // dS^T_i in shared memory (EW_THREADS)
     uint64_t *bar_dqe = bar_dsf + 1;       // dQ_i read out of TMEM (EW_THREADS)
     uint64_t *bar_stg = bar_dqe + 1;       // dQ_i staged over Q_i and dO_i (EW_THREADS)
     uint64_t *bar_done = bar_stg + 1;
-    static_assert(C::NBARS >= 1 + QSL + OSL + 10, "barrier slots");
+    static_assert(C::NBARS >= 1 + QSL + OSL + 11, "barrier slots");
     uint32_t *tmem_slot = (uint32_t *)(bars + C::NBARS);
     volatile int *abort = (volatile int *)(tmem_slot + 1);
 
@@ -874,6 +875,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NBARS; ++i) mbar_init(&bars[i], 1);
         mbar_init(bar_ptf, EW_THREADS);
+        mbar_init(bar_dpr, EW_THREADS);
         mbar_init(bar_dsf, EW_THREADS);
         mbar_init(bar_dqe, EW_THREADS);
         mbar_init(bar_stg, EW_THREADS);
@@ -1021,12 +1023,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (ok) ok = issue_dpt(0);
                 for (int i = 0; ok && i < nsteps; ++i) {
                     ok = issue_dv(i);
+                    // S^T_{i+1} overwrites dP^T_i as soon as the element-wise warps have
+                    // read it: the tensor pipe runs it while they form and store dS^T_i
+                    if (ok) ok = mbar_wait(bar_dpr, i & 1, abort);
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (i + 1 < nsteps) ok = issue_st(i + 1);
                     if (ok) ok = mbar_wait(bar_dsf, i & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    // S^T_{i+1} overwrites dP^T_i, which the element-wise warps have read
-                    if (i + 1 < nsteps) ok = issue_st(i + 1);
-                    if (!ok) break;
                     issue_dk_dq(i);
                     if (i + 1 < nsteps) {
                         ok = mbar_wait(bar_dqe, i & 1, abort);
@@ -1050,40 +1055,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         constexpr int HC = BM / EW;  // rows per thread and step
         constexpr int DC = D / EW;   // dQ columns per thread
-        float *r_lse = reinterpret_cast<float *>(smem + C::OFF_ROW);  // exp2 domain
-        float *r_d = r_lse + BM;
-        int *r_lo = reinterpret_cast<int *>(r_d + BM);
-        int *r_hi = r_lo + BM;
-        int *r_full = r_hi + BM;  // [0] largest lo, [1] smallest hi of the step
-        // Row data of a step (lse, D_t, the row's key interval, and the step's
-        // fully visible key range), gathered by threads 0..127 a step ahead.
-        struct RowData {
-            float L, dd;
-            int lo, hi, flo, fhi;
+        // the query rows that see key s: one interval (empty for keys past Tk)
+        int ta, tb;
+        key_rows(P.mask, s, ta, tb);
+        // Row data of step j in slot j & 1: lse and D_t of its rows and the rows
+        // [t0, t1] themselves.  Threads 0..127 fill a step's slot one step ahead with
+        // asynchronous copies, so no thread waits on a global load inside the loop.
+        struct RowSlot {
+            float lse[BM], d[BM];
+            int t0, t1, pad[2];
         };
-        auto gather = [&](int i) -> RowData {
-            RowData d{-INFINITY, 0.f, 1, 0, 1, 0};
-            if (tid >= BM || i >= nsteps) return d;
+        static_assert(sizeof(RowSlot) == C::ROW_BYTES, "row slot layout");
+        RowSlot *slots = reinterpret_cast<RowSlot *>(smem + C::OFF_ROW);
+        auto prefetch = [&](int j) {
+            if (tid >= BM || j >= nsteps) return;
+            RowSlot &rs = slots[j & 1];
             int t0, t1;
-            slice(i, t0, t1);
+            slice(j, t0, t1);
             const int t = t0 + tid;
             if (t <= t1) {
-                if (row_interval(P.mask, t, d.lo, d.hi) != 0) { d.lo = 1; d.hi = 0; }
-                d.L = __ldg(lse + ((int64_t)b * P.H + h) * P.Tq + t);
-                d.dd = __ldg(Dws + ((int64_t)b * P.H + h) * P.Tq + t);
+                const int64_t o = ((int64_t)b * P.H + h) * P.Tq + t;
+                cp_async_4(&rs.lse[tid], lse + o);
+                cp_async_4(&rs.d[tid], Dws + o);
+                cp_async_commit();
+            } else {  // a row past the slice: never visible, D_t must stay finite
+                rs.lse[tid] = 0.f;
+                rs.d[tid] = 0.f;
             }
             if (tid == 0) {
-                // every row of the step valid: the interval ends are monotone, so the
-                // step is fully visible to keys in [lo(last row), hi(first row)]
-                const int tl_ = t0 + BM - 1;
-                int lo1 = 1, hi1 = 0, lo0 = 1, hi0 = 0;
-                if (tl_ <= t1 && row_interval(P.mask, tl_, lo1, hi1) == 0 &&
-                    row_interval(P.mask, t0, lo0, hi0) == 0) {
-                    d.flo = lo1;
-                    d.fhi = hi0;
-                }
+                rs.t0 = t0;
+                rs.t1 = t1;
             }
-            return d;
         };
         // dQ_j: TMEM -> registers -> the swizzled boxes of tm_dq over the slots
         // of Q_j and dO_j (no product reads them once dQ_j is complete); the
@@ -1109,26 +1111,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_arrive(bar_stg);
             return true;
         };
-        RowData next = gather(0);
+        prefetch(0);
         bool ok = !skip;
         for (int i = 0; i < nsteps; ++i) {
-            if (i > 0) ew_sync();  // every thread is done with step i-1's row data
-            if (ok && tid < BM) {
-                r_lse[tid] = (next.L == -INFINITY) ? INFINITY : next.L * 1.4426950408889634f;
-                r_d[tid] = next.dd;
-                r_lo[tid] = next.lo;
-                r_hi[tid] = next.hi;
-                if (tid == 0) {
-                    r_full[0] = next.flo;
-                    r_full[1] = next.fhi;
-                }
-            }
-            next = gather(i + 1);
-            // row data written; all element-wise warps agree to go on.  A warp whose
-            // wait fails below skips to the next iteration, where every warp stops
-            // here (the named barriers of an iteration all sit before its waits).
+            cp_async_wait_all();  // this thread's copies into slot i & 1 have landed
+            // Slot i & 1 complete and visible, every thread done with step i-1 (whose
+            // slot the next prefetch overwrites), and all element-wise warps agree to go
+            // on.  A warp whose wait fails below skips to the next iteration, where
+            // every warp stops here (the only named barrier of an iteration).
             ok = group_all(ok);
             if (!ok) break;
+            prefetch(i + 1);
+            const RowSlot &rs = slots[i & 1];
+            // this thread's rows: tr0 .. tr0 + HC - 1, visible while in [ta, tmax]
+            const int tr0 = rs.t0 + eg * HC;
+            const int tmax = min(tb, rs.t1);
             // ---- P^T_i = exp(S^T_i scale - lse) over region(i)
             ok = __all_sync(0xffffffffu, mbar_wait(bar_sf, i & 1, abort));
             if (!ok) continue;
@@ -1136,18 +1133,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t v[HC];
             tmem_ldn<HC>(tl + region(i) + eg * HC, v);
             tmem_ld_wait();
-            const bool full = r_full[0] <= s && s <= r_full[1];
-            const float *cl = r_lse + eg * HC;
+            const float *cl = rs.lse + eg * HC;
             float p[HC];
-            if (full) {
+            if (ta <= tr0 && tr0 + HC - 1 <= tmax) {
 #pragma unroll
-                for (int r = 0; r < HC; ++r) p[r] = ex2(fmaf(__uint_as_float(v[r]), sl2, -cl[r]));
+                for (int r = 0; r < HC; ++r)
+                    p[r] = ex2(fmaf(__uint_as_float(v[r]), sl2, -1.4426950408889634f * cl[r]));
             } else {
-                const int *clo = r_lo + eg * HC, *chi = r_hi + eg * HC;
+                // a visible row has a finite lse; the others take 0 without using theirs
 #pragma unroll
                 for (int r = 0; r < HC; ++r) {
-                    const bool vis = (clo[r] <= s) && (s <= chi[r]);
-                    p[r] = vis ? ex2(fmaf(__uint_as_float(v[r]), sl2, -cl[r])) : 0.f;
+                    const bool vis = ta <= tr0 + r && tr0 + r <= tmax;
+                    const float e = ex2(fmaf(__uint_as_float(v[r]), sl2, -1.4426950408889634f * cl[r]));
+                    p[r] = vis ? e : 0.f;
                 }
             }
             {
@@ -1170,7 +1168,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             tmem_ldn<HC>(tl + region(i + 1) + eg * HC, v);
             tmem_ld_wait();
-            const float *cd = r_d + eg * HC;
+            tc_fence_before();
+            mbar_arrive(bar_dpr);  // region(i + 1) may take S^T_{i+1}
+            const float *cd = rs.d + eg * HC;
 #pragma unroll
             for (int r = 0; r < HC; ++r) p[r] = p[r] * (__uint_as_float(v[r]) - cd[r]);
             // at D = 128 the tile is dO_i's slot: dV_i must have read it
@@ -1190,10 +1190,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 u.w = pack_bf16(p[8 * j + 6], p[8 * j + 7]);
                 *reinterpret_cast<uint4 *>(ds_tile + sw128_offset(sl, eg * (HC / 8) + j, BN)) = u;
             }
-            tc_fence_before();        // dP^T_i read: region(i + 1) may take S^T_{i+1}
             fence_proxy_async_smem();  // dS^T_i visible to the tensor pipe
             mbar_arrive(bar_dsf);
         }
+        cp_async_wait_all();  // no copy outlives the loop
         if (ok && nsteps > 0) ok = write_dq(nsteps - 1);
         // ------------------------------------------------------ epilogue ---
         // each warpgroup writes a quarter of the D columns of its keys' dV and dK
