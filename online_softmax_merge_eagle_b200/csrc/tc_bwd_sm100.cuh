@@ -735,16 +735,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 // product reads once dQ_i is complete: the element-wise warps stage it there
 // (fp32, in the swizzled boxes of a TMA tensor map over the accumulator), and
 // the producer warp, which owns the slots, issues TMA reduce-adds (whole L2
-// lines), waits until they have read the slots and then loads dO_{i+2} and
-// Q_{i+3} into them -- a step and two steps before they are needed, so the
-// reductions drain while the next steps compute.
+// lines) in two bulk groups, the boxes over dO_i's slot first, and loads
+// dO_{i+2} as soon as that group has read its slot and Q_{i+3} once the second
+// has -- a step and two steps before they are needed, so the reductions drain
+// while the next steps compute.
 // TMEM: dV [0, D), dK [128, 128 + D) and two 128-column regions R0, R1 that
 // carry in turn S^T_i -> P^T_i (R_{i%2}), dP^T_i (R_{(i+1)%2}) and dQ_i
 // (R_{i%2}, issued after dV_i has read P^T_i).
-// MMA issue order: S^T_0, dP^T_0, then per step i: dV_i (once P^T_i is
-// written); S^T_{i+1}, dK_i, dQ_i (once dS^T_i is in shared memory);
-// dP^T_{i+1} (once the element-wise warps have read dQ_i out of R_{i%2}).
-// Element-wise order per step: P^T_i, then dQ_{i-1} out, then dS^T_i.
+// MMA issue order: S^T_0, dP^T_0, dV_0, then per step i: S^T_{i+1} (once the
+// element-wise warps have read dP^T_i); dK_i, dQ_i (once dS^T_i is in shared
+// memory); dV_{i+1} (once P^T_{i+1} is written); dP^T_{i+1} (once dQ_i has
+// been read out of R_{i%2}).  The elementwise warps' order per step: P^T_i,
+// then dQ_{i-1} out, then dP^T_i read and dS^T_i.
 namespace kvq {
 
 constexpr int BN = 128;  // keys per CTA (TMEM lanes of S^T, dP^T, dV, dK)
@@ -932,14 +934,23 @@ __global__ void __launch_bounds__(THREADS, 1)
                 int t0, t1;
                 slice(i, t0, t1);
                 const int row0 = (b * P.H + h) * P.Tq + t0;
+                // the boxes over dO_i's slot as one bulk group, then those over Q_i's:
+                // dO_{i+2}, needed first, goes in as soon as its slot has been read
 #pragma unroll
-                for (int bx = 0; bx < C::NBOX; ++bx)
+                for (int bx = C::NBOX / 2; bx < C::NBOX; ++bx)
                     tma_reduce_add_2d(&tm_dq, smem + C::box_off(i, bx), bx * DQ_BOX_COLS, row0);
                 bulk_commit();
-                if (i + OSL < nsteps || i + QSL < nsteps) {
-                    bulk_wait_read_all();  // the slots are free again
-                    if (i + OSL < nsteps) load(true, o_issued++);
-                    if (i + QSL < nsteps) load(false, q_issued++);
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX / 2; ++bx)
+                    tma_reduce_add_2d(&tm_dq, smem + C::box_off(i, bx), bx * DQ_BOX_COLS, row0);
+                bulk_commit();
+                if (i + OSL < nsteps) {
+                    bulk_wait_read_but_newest();  // dO_i's slot is free again
+                    load(true, o_issued++);
+                }
+                if (i + QSL < nsteps) {
+                    bulk_wait_read_all();  // and Q_i's
+                    load(false, q_issued++);
                 }
             }
             bulk_wait_all();  // every reduce-add has landed
@@ -1018,14 +1029,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                             sdesc_sw128(k_s + kk * 2048, BN * 128, 1024), id_dq, kk > 0 ? 1u : 0u);
                 umma_commit(bar_dqf);
             };
+            // Per step i the pipe runs S^T_{i+1}, dK_i + dQ_i, dV_{i+1}, dP^T_{i+1}:
+            // S^T_{i+1} overwrites dP^T_i as soon as the element-wise warps have read
+            // it (they form and store dS^T_i meanwhile), and dV_{i+1} runs while they
+            // read dQ_i out of the region dP^T_{i+1} takes next.
             if (ok && nsteps > 0) {
                 ok = issue_st(0);
                 if (ok) ok = issue_dpt(0);
+                if (ok) ok = issue_dv(0);
                 for (int i = 0; ok && i < nsteps; ++i) {
-                    ok = issue_dv(i);
-                    // S^T_{i+1} overwrites dP^T_i as soon as the element-wise warps have
-                    // read it: the tensor pipe runs it while they form and store dS^T_i
-                    if (ok) ok = mbar_wait(bar_dpr, i & 1, abort);
+                    ok = mbar_wait(bar_dpr, i & 1, abort);
                     if (!ok) break;
                     tc_fence_after();
                     if (i + 1 < nsteps) ok = issue_st(i + 1);
@@ -1034,7 +1047,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc_fence_after();
                     issue_dk_dq(i);
                     if (i + 1 < nsteps) {
-                        ok = mbar_wait(bar_dqe, i & 1, abort);
+                        // dV_{i+1} reads dO_{i+1}, which no product has waited for yet
+                        ok = mbar_wait(bar_of + (i + 1) % OSL, ((i + 1) / OSL) & 1, abort);
+                        if (ok) ok = issue_dv(i + 1);
+                        if (ok) ok = mbar_wait(bar_dqe, i & 1, abort);
                         if (ok) ok = issue_dpt(i + 1);
                     }
                 }
