@@ -135,6 +135,21 @@ EAGLE_HD void key_rows(const MaskDesc &m, int s, int &ta, int &tb) {
     keys_row_range(m, s, s, ta, tb);
 }
 
+// Block order of the tile kernels.  Blocks start in increasing linear index, so
+// the tile index (0 = the tile with the most steps under the causal masks) is made
+// the slow index within groups of HEAVY_GROUP (batch, head) pairs: a group's
+// heaviest tiles start first and its lightest end it, which keeps the last wave
+// short, while only the group's pairs share L2.  lin = the block's linear index
+// over a grid of ntiles x npairs blocks; returns its tile and pair (b * H + h).
+constexpr int HEAVY_GROUP = 8;
+EAGLE_HD void heavy_first(int lin, int ntiles, int npairs, int &tile, int &pair) {
+    const int first = lin / (HEAVY_GROUP * ntiles) * HEAVY_GROUP;  // the group's first pair
+    const int gs = npairs - first < HEAVY_GROUP ? npairs - first : HEAVY_GROUP;
+    const int idx = lin - first * ntiles;
+    tile = idx / gs;
+    pair = first + idx % gs;
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {

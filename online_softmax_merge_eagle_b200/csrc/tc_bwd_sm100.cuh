@@ -161,7 +161,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ks = blockIdx.x * BN, h = blockIdx.y, b = blockIdx.z;
+    int kt, pr;  // grid (key tiles, H, B), heaviest key tiles first
+    heavy_first(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), gridDim.x,
+                gridDim.y * gridDim.z, kt, pr);
+    const int ks = kt * BN, h = pr % gridDim.y, b = pr / gridDim.y;
     int tbeg, tend;
     keys_row_range(P.mask, ks, min(ks + BN, P.Tk) - 1, tbeg, tend);
     const int nsteps = tend >= tbeg ? (tend - tbeg + BM) / BM : 0;
@@ -480,8 +483,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_qtiles = (P.Tq + BM - 1) / BM;
-    const int t0 = (n_qtiles - 1 - (int)blockIdx.x) * BM;  // heaviest causal tiles first
-    const int h = blockIdx.y, b = blockIdx.z;
+    int qt, pr;  // grid (query tiles, H, B), heaviest (last) query tiles first
+    heavy_first(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), gridDim.x,
+                gridDim.y * gridDim.z, qt, pr);
+    const int t0 = (n_qtiles - 1 - qt) * BM;
+    const int h = pr % gridDim.y, b = pr / gridDim.y;
     int kbeg, kend;
     rows_key_range(P.mask, t0, min(t0 + BM, P.Tq) - 1, kbeg, kend);
     const int nsteps = kend >= kbeg ? (kend - kbeg + BN) / BN : 0;
@@ -831,7 +837,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int *abort = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ks = blockIdx.x * BN, h = blockIdx.y, b = blockIdx.z;
+    int kt, pr;  // grid (key tiles, H, B), heaviest key tiles first
+    heavy_first(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z), gridDim.x,
+                gridDim.y * gridDim.z, kt, pr);
+    const int ks = kt * BN, h = pr % gridDim.y, b = pr / gridDim.y;
     int tbeg, tend;
     keys_row_range(P.mask, ks, min(ks + BN, P.Tk) - 1, tbeg, tend);
     // query slices: 128 rows at a time from tbeg or, with a q_tiles list, the

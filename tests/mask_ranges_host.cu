@@ -6,6 +6,7 @@
 //   Q t0 t1 kbeg kend      rows_key_range for rows [t0, t1] (several tile lengths)
 //   K k0 k1 tbeg tend      keys_row_range for keys [k0, k1] (several tile lengths)
 //   S s ta tb              key_rows for every key s in [-1, Tk]
+//   G nt np lin tile pair  heavy_first over grids of nt tiles x np (batch, head) pairs
 #include <cstdio>
 #include <vector>
 
@@ -52,5 +53,12 @@ int main() {
         eagle::key_rows(m, s, a, b);
         printf("S %d %d %d\n", s, a, b);
     }
+    const int grids[6][2] = {{1, 1}, {5, 19}, {64, 64}, {3, 8}, {7, 9}, {2, 17}};
+    for (int g = 0; g < 6; ++g)
+        for (int lin = 0; lin < grids[g][0] * grids[g][1]; ++lin) {
+            int tile, pair;
+            eagle::heavy_first(lin, grids[g][0], grids[g][1], tile, pair);
+            printf("G %d %d %d %d %d\n", grids[g][0], grids[g][1], lin, tile, pair);
+        }
     return 0;
 }

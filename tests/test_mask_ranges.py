@@ -91,7 +91,7 @@ def test_mask_ranges_match_brute_force(driver, case):
     Tq, Tk, q_off, k_off, causal, cu = CASES[case]
     vis = visibility(Tq, Tk, q_off, k_off, causal, cu)
     lines = run(driver, Tq, Tk, q_off, k_off, causal, cu)
-    n = {"R": 0, "Q": 0, "K": 0, "S": 0}
+    n = {"R": 0, "Q": 0, "K": 0, "S": 0, "G": 0}
     last_cls = -1
     for rec in lines:
         kind, vals = rec[0], [int(x) for x in rec[1:]]
@@ -113,8 +113,29 @@ def test_mask_ranges_match_brute_force(driver, case):
             k0, k1, a, b = vals
             sp = span(vis[:, k0:k1 + 1].any(axis=1))
             assert (b < a) if sp is None else ((a, b) == sp), rec
-        else:
+        elif kind == "S":
             s, a, b = vals
             sp = span(vis[:, s]) if 0 <= s < Tk else None
             assert (b < a) if sp is None else ((a, b) == sp), rec
     assert n["R"] == Tq and n["S"] == Tk + 2 and n["Q"] > 0 and n["K"] > 0
+
+
+def test_block_order_is_a_grouped_heaviest_first_bijection(driver):
+    """heavy_first maps the blocks of a (tiles x pairs) grid one to one onto
+    (tile, pair); within each group of 8 consecutive pairs the tile index never
+    decreases with the block's linear index, so a group's heaviest tiles start
+    first."""
+    lines = [r for r in run(driver, *CASES["causal"]) if r[0] == "G"]
+    grids = {}
+    for rec in lines:
+        nt, npairs, lin, tile, pair = (int(x) for x in rec[1:])
+        grids.setdefault((nt, npairs), []).append((lin, tile, pair))
+    assert len(grids) == 6
+    for (nt, npairs), recs in grids.items():
+        assert sorted(r[0] for r in recs) == list(range(nt * npairs))
+        assert sorted((t, p) for _, t, p in recs) == [(t, p) for t in range(nt) for p in range(npairs)]
+        last = {}
+        for lin, tile, pair in sorted(recs):
+            group = pair // 8
+            assert tile >= last.get(group, 0), (nt, npairs, lin)
+            last[group] = tile
