@@ -14,19 +14,26 @@ merged once at the end (_merge_diag), before the cast to q's dtype.
 
 The backward ("eagle.zigzag_ring_attention", zigzag_ring_flash_attn_varlen_
 backward) runs every such pair against the FINAL merged out / lse of the
-query rows.  dQ accumulates locally; the dK / dV of a block-0 shard travel with
-it, in fp32, and make the whole circle (cp hops), so that every rank's
-accumulator comes home holding the contributions of all ranks.  The diagonal
-blocks' gradients are local and closed form; they come with the pairs on the
-diagonal.
+query rows.  dQ accumulates locally; the dK / dV running sums of a block-0
+shard travel the ring one step behind its K/V, in fp32, and make the whole
+circle (cp hops), so that every rank's sum comes home holding the
+contributions of all ranks.  A rank computes its contribution to the visiting
+shard into a zeroed buffer while that shard's running sum is still in flight
+from the previous rank, and adds it on arrival before passing the sum on: the
+hop overlaps the step's compute.  The diagonal blocks' gradients are local and
+closed form; they come with the pairs on the diagonal.
 
 Every compute step is one of five operations (``ops``): the default,
 ``LIBRARY_OPS``, calls libeagleattn (eagle_attn_fwd / eagle_attn_bwd with
 global offsets, attn_merge_out_lse, attn_merge_diag, attn_finalize); a caller
 may pass another object with the same five methods.  Communication is
 torch.distributed point-to-point (batch_isend_irecv: NCCL over NVLink between
-GPUs, or any backend that supports it); the forward's K/V exchange is posted
-before the step's compute, so that the transfer overlaps it.
+GPUs, or any backend that supports it); the K/V exchange is posted before the
+step's compute, so that the transfer overlaps it.  Between two ranks the
+messages of the two streams (K/V, and the backward's running sums) are posted
+in the same order on both sides: every rank posts a step's receive of a
+running sum before that step's K/V exchange and sends its updated sum after
+the step's compute.
 """
 from __future__ import annotations
 
@@ -118,7 +125,7 @@ def _exchange(send: list[torch.Tensor], recv: list[torch.Tensor], nxt: int, prv:
     from the previous one; returns the works to wait on."""
     ops = [dist.P2POp(dist.isend, t, nxt, group) for t in send]
     ops += [dist.P2POp(dist.irecv, t, prv, group) for t in recv]
-    return dist.batch_isend_irecv(ops)
+    return dist.batch_isend_irecv(ops) if ops else []
 
 
 def _pairs(r: int, src: int, cp: int):
@@ -190,19 +197,35 @@ def ring_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, group=N
     r, cp, nxt, prv = _ring(group)
     f32 = dict(dtype=torch.float32, device=q.device)
     dq32 = torch.zeros(q.shape, **f32)
-    dk32 = torch.zeros(cache_k.shape, **f32)  # this shard's blocks; block 0 travels
+    dk32 = torch.zeros(cache_k.shape, **f32)  # this shard's blocks (block 0: its own part first)
     dv32 = torch.zeros(cache_k.shape, **f32)
     lse_c = [lse[:, :, qi * c:(qi + 1) * c].contiguous() for qi in range(2)]
     kv = [cache_k[:, :1].contiguous(), cache_v[:, :1].contiguous()]
-    own = [dk32[:, :1], dv32[:, :1]]  # this shard's block-0 accumulators
-    acc = own                         # the accumulators of the visiting shard
     kv_next = [torch.empty_like(kv[0]), torch.empty_like(kv[1])] if cp > 1 else None
-    spare = [[torch.empty((1, 1, T2, H, D), **f32) for _ in range(2)] for _ in range(2)] \
+    acc_shape = (1, 1, T2, H, D)
+    # this rank's part of the visiting shard's block-0 dK / dV (steps s >= 1), and
+    # two buffers for the running sums that arrive, one per step parity: a sum is
+    # received, completed and sent on from the same buffer
+    part = [torch.empty(acc_shape, **f32) for _ in range(2)] if cp > 1 else None
+    inbox = [[torch.empty(acc_shape, **f32) for _ in range(2)] for _ in range(2)] \
         if cp > 1 else None
-    acc_next = spare[0] if cp > 1 else None
+    sending = [[], []]  # the works of the send out of inbox[0] / inbox[1] (or of step 0)
     for s in range(cp):
         src = (r - s) % cp
+        # the running sum of shard src (the previous rank's step s-1), then this step's K/V
+        box = inbox[s & 1] if s > 0 else None
+        if s > 0:
+            for w in sending[s & 1]:  # the buffer's last send has left it
+                w.wait()
+            sending[s & 1] = []
+        recv_works = _exchange([], box, nxt, prv, group) if s > 0 else []
         works = _exchange(kv, kv_next, nxt, prv, group) if s + 1 < cp else []
+        if s == 0:
+            acc = [dk32[:, :1], dv32[:, :1]]
+        else:
+            for t in part:
+                t.zero_()
+            acc = part
         for qi, qc, ki, kc in _pairs(r, src, cp):
             qrows = slice(qi * c, (qi + 1) * c)
             krows = slice(ki * c, (ki + 1) * c)
@@ -218,17 +241,27 @@ def ring_zigzag_backward(grad_out, q, cache_k, cache_v, out, lse, scale, group=N
         for w in works:
             w.wait()
         if cp > 1:
-            # the accumulators move on with their K/V: the own ones leave after
-            # step 0 and come back after the last step
-            for w in _exchange([a.contiguous() for a in acc], acc_next, nxt, prv, group):
-                w.wait()
-            acc, acc_next = acc_next, (spare[1] if acc is own else acc)
+            if s == 0:
+                out_sum = acc  # this shard's own part starts its circle
+            else:
+                for w in recv_works:
+                    w.wait()
+                box[0].add_(part[0])
+                box[1].add_(part[1])
+                out_sum = box
+            sending[s & 1] = _exchange(out_sum, [], nxt, prv, group)
             if s + 1 < cp:
                 kv, kv_next = kv_next, kv
     if cp > 1:
-        # after cp hops the accumulators of this rank's own shard are home
-        dk32[:, :1].copy_(acc[0])
-        dv32[:, :1].copy_(acc[1])
+        # after cp hops the running sums of this rank's own shard are home
+        home = [torch.empty(acc_shape, **f32) for _ in range(2)]
+        for w in _exchange([], home, nxt, prv, group):
+            w.wait()
+        for ws in sending:
+            for w in ws:
+                w.wait()
+        dk32[:, :1].copy_(home[0])
+        dv32[:, :1].copy_(home[1])
     dq = torch.empty_like(q)
     dk = torch.empty_like(cache_k)
     dv = torch.empty_like(cache_v)
