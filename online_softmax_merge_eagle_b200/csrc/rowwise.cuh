@@ -458,7 +458,16 @@ __global__ void __launch_bounds__(ROW_THREADS) dq_finalize_kernel(Problem P,
     const int64_t idx = (int64_t)blockIdx.x * (ROW_THREADS / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     int b, t, h;
-    if (!row_of(P, idx, b, t, h)) return;
+    if (!P.q_tiles) {
+        // rows in the accumulator's order (b, h, t): consecutive warps read
+        // consecutive accumulator rows, the larger of the two streams
+        if (idx >= (int64_t)P.B * P.H * P.Tq) return;
+        t = (int)(idx % P.Tq);
+        h = (int)((idx / P.Tq) % P.H);
+        b = (int)(idx / ((int64_t)P.H * P.Tq));
+    } else if (!row_of(P, idx, b, t, h)) {
+        return;
+    }
     const int64_t qo = b * P.q_sb + t * P.q_st + (int64_t)h * P.D + lane * E;
     const int64_t li = ((int64_t)b * P.H + h) * P.Tq + t;
     float a[E];
