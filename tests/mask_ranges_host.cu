@@ -1,4 +1,4 @@
-// Host driver for the library's mask range functions (common.cuh), built and run
+// Host harness for the library's mask range functions (common.cuh), built and run
 // by tests/test_mask_ranges.py.  Reads one mask from stdin:
 //   Tq Tk q_off k_off causal num_docs cu[0] .. cu[num_docs]   (num_docs = 0: no documents)
 // and prints, one line each,

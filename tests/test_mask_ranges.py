@@ -20,9 +20,9 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 
 @pytest.fixture(scope="module")
-def driver(tmp_path_factory):
+def harness(tmp_path_factory):
     if not os.path.exists(NVCC) and shutil.which("nvcc") is None:
-        pytest.fail("nvcc is needed to build the host driver of the mask functions")
+        pytest.fail("nvcc is needed to build the host harness of the mask functions")
     exe = str(tmp_path_factory.mktemp("mask") / "mask_ranges")
     subprocess.check_call([NVCC if os.path.exists(NVCC) else "nvcc", "-std=c++17", "-O1",
                            "-gencode", "arch=compute_100a,code=sm_100a",
@@ -58,12 +58,12 @@ def span(mask_1d):
     return int(idx[0]), int(idx[-1])
 
 
-def run(driver, Tq, Tk, q_off, k_off, causal, cu):
+def run(harness, Tq, Tk, q_off, k_off, causal, cu):
     nd = 0 if cu is None else len(cu) - 1
     text = f"{Tq} {Tk} {q_off} {k_off} {int(causal)} {nd}"
     if cu is not None:
         text += " " + " ".join(str(int(x)) for x in cu)
-    out = subprocess.run([driver], input=text, capture_output=True, text=True, check=True).stdout
+    out = subprocess.run([harness], input=text, capture_output=True, text=True, check=True).stdout
     return [line.split() for line in out.splitlines()]
 
 
@@ -87,10 +87,10 @@ CASES = {
 
 
 @pytest.mark.parametrize("case", sorted(CASES))
-def test_mask_ranges_match_brute_force(driver, case):
+def test_mask_ranges_match_brute_force(harness, case):
     Tq, Tk, q_off, k_off, causal, cu = CASES[case]
     vis = visibility(Tq, Tk, q_off, k_off, causal, cu)
-    lines = run(driver, Tq, Tk, q_off, k_off, causal, cu)
+    lines = run(harness, Tq, Tk, q_off, k_off, causal, cu)
     n = {"R": 0, "Q": 0, "K": 0, "S": 0, "G": 0}
     last_cls = -1
     for rec in lines:
@@ -120,12 +120,12 @@ def test_mask_ranges_match_brute_force(driver, case):
     assert n["R"] == Tq and n["S"] == Tk + 2 and n["Q"] > 0 and n["K"] > 0
 
 
-def test_block_order_is_a_grouped_heaviest_first_bijection(driver):
+def test_block_order_is_a_grouped_heaviest_first_bijection(harness):
     """heavy_first maps the blocks of a (tiles x pairs) grid one to one onto
     (tile, pair); within each group of 8 consecutive pairs the tile index never
     decreases with the block's linear index, so a group's heaviest tiles start
     first."""
-    lines = [r for r in run(driver, *CASES["causal"]) if r[0] == "G"]
+    lines = [r for r in run(harness, *CASES["causal"]) if r[0] == "G"]
     grids = {}
     for rec in lines:
         nt, npairs, lin, tile, pair = (int(x) for x in rec[1:])

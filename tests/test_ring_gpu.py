@@ -1,6 +1,5 @@
 """The sequence-parallel zig-zag ring (NeMo AutoModel "eagle.zigzag_ring_attention")
-through libeagleattn on one GPU.  A run of this pool gets one GPU, so the ring
-has one rank here: its shard is the whole sequence as two chunks and no shard
+through libeagleattn on one GPU.  With one GPU the ring has one rank: its shard is the whole sequence as two chunks and no shard
 moves, but every compute step (block forward with global offsets, merges, the
 diagonal merge, the per-pair backward into fp32 accumulators, the casts) is the
 library's, checked against the fp64 oracle.  The exchange between ranks is
