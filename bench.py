@@ -52,8 +52,10 @@ def visible_pairs(w) -> int:
     qp = w.q_pos_offset + t
     if w.doc_lengths is not None:
         cu = np.concatenate([[0], np.cumsum(w.doc_lengths)]).astype(np.int64)
-        d = np.searchsorted(cu, qp, side="right") - 1
-        glo, ghi = cu[d], cu[d + 1] - 1
+        d = np.clip(np.searchsorted(cu, qp, side="right") - 1, 0, len(cu) - 2)
+        inside = (qp >= 0) & (qp < cu[-1])  # rows outside every document see nothing
+        glo = np.where(inside, cu[d], 1 << 60)
+        ghi = np.where(inside, cu[d + 1] - 1, -(1 << 60))
     else:
         glo = np.full_like(qp, -(1 << 60))
         ghi = np.full_like(qp, 1 << 60)
