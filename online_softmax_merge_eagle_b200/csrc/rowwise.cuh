@@ -378,8 +378,11 @@ __global__ void __launch_bounds__(ROW_THREADS) bwd_diag_kernel(
 // (added to what the buffers hold).  With zero_dq, dq_diag is written (zeros)
 // also when there are no diagonal blocks.  With a q_tiles list, the listed rows
 // only.
+// Eight blocks (64 warps) per SM when the gradients are bf16: the row pass is
+// bound by the loads each SM keeps in flight, and 32 registers leave room for
+// all of them (the fp32-gradient form would spill there).
 template <typename T, typename TO, typename GT, int E>
-__global__ void __launch_bounds__(ROW_THREADS) bwd_rows_kernel(
+__global__ void __launch_bounds__(ROW_THREADS, sizeof(GT) == 2 ? 8 : 1) bwd_rows_kernel(
     Problem P, const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const T *__restrict__ dout, const TO *__restrict__ out, const float *__restrict__ lse,
     float *__restrict__ Dws, float *__restrict__ dq_diag, GT *__restrict__ dk,
