@@ -70,9 +70,10 @@ constexpr int MERGE_U = 2;          // rows per lane in flight
 // (32 / (D/4) rows per warp instruction), MERGE_U rows in flight per lane.
 // Grid: (H, ceil(T / (4 * 32)), B), the head fastest: the rows of all heads of a
 // t range are adjacent in memory, so the blocks in flight together read whole
-// DRAM pages instead of one head's slice of many.
+// DRAM pages instead of one head's slice of many.  Twelve blocks per SM (40
+// registers): more rows in flight per SM than the nine the unbounded form fits.
 template <typename TB, int D4>
-__global__ void __launch_bounds__(MERGE_THREADS) merge_kernel(float *__restrict__ out,
+__global__ void __launch_bounds__(MERGE_THREADS, 12) merge_kernel(float *__restrict__ out,
                                                              float *__restrict__ lse,
                                                              const TB *__restrict__ bout,
                                                              const float *__restrict__ blse,
